@@ -1,0 +1,442 @@
+"""Benchmark: one decode step of packed-KV attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+Workload (the decode GQA configuration): batch 32, H_q 32, H_kv 8, d_h 128,
+context 4096 for every sequence, 4-bit codes in groups of 32 with float32
+scales, bf16 Q and O.  One step is one pass of the whole hot path for a
+decode step:
+
+  1. append -- kvq_pack re-packs the tail K group (tokens 4064..4095, where
+     the new token sits) and the V rows of those tokens from a float32
+     recent-token window, and
+  2. attend -- kvq_attend over the whole 4096-token packed cache.
+
+Two independent packed caches (2 x 168 MB, more than the 126 MB L2) are used
+in turn so no step reads the previous step's cache from L2.
+
+Prints one JSON line (rank 0).  ``value`` is algorithmic bytes per step
+(packed codes + scales of every valid token + Q + O for the attend, float32
+window in + codes/scales out for the append) over the device time per step,
+summed over all ranks and divided by the max over ranks.
+
+``--impl reference`` times the CPU oracle instead (NumPy, on this host's
+cores), on a bounded sample of the same workload, and reports the same
+metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "4-bit packed-KV attention: achieved HBM GB/s (% of 8 TB/s), µs per decode step"
+WORKLOAD = "decode_gqa"
+SEED = 0
+
+
+# ---------------------------------------------------------------------------
+# byte accounting
+# ---------------------------------------------------------------------------
+
+def attend_bytes(B, H_q, H_kv, D, lengths, bits=4, group=32, q_bytes=2, o_bytes=2, lq=1):
+    """Algorithmic bytes of one attend: codes + scales of every valid token of
+    every (b, h_kv), plus Q and O.  K scales count per started group of g
+    tokens (a K group's scale row is read whole), V scales per token."""
+    dp = -(-D // group) * group
+    total = 0
+    for n in lengths:
+        n = int(n)
+        k_codes = n * D * bits // 8
+        v_codes = n * dp * bits // 8
+        k_scales = -(-n // group) * D * 4
+        v_scales = n * (dp // group) * 4
+        total += H_kv * (k_codes + v_codes + k_scales + v_scales)
+    total += B * H_q * lq * D * (q_bytes + o_bytes)
+    return total
+
+
+def append_bytes(B, H_kv, D, tokens, bits=4, group=32, in_bytes=4):
+    dp = -(-D // group) * group
+    per_head = (2 * tokens * D * in_bytes                     # K, V window in
+                + tokens * D * bits // 8 + tokens * dp * bits // 8   # codes out
+                + -(-tokens // group) * D * 4 + tokens * (dp // group) * 4)  # scales out
+    return B * H_kv * per_head
+
+
+# ---------------------------------------------------------------------------
+# environment
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def recorded_traffic(kernel_src: str):
+    """Per-launch DRAM bytes of the attend kernel from the committed ncu
+    summary, or None when the kernel source changed since the capture."""
+    import hashlib
+    summary = os.path.join(ROOT, "profiles", "attend_decode_gqa_b32_ctx4096.md")
+    try:
+        text = open(summary, encoding="utf-8").read()
+        src = open(kernel_src, "rb").read()
+    except OSError:
+        return None
+    digest = hashlib.sha256(src).hexdigest()[:16]
+    want, traffic = None, None
+    for line in text.splitlines():
+        if line.startswith("kernel_source_sha256_16:"):
+            want = line.split(":", 1)[1].strip()
+        if line.startswith("dram_bytes_per_launch:"):
+            traffic = int(line.split(":", 1)[1].strip().replace(",", ""))
+    return traffic if (want == digest and traffic) else None
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML on a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: clocks reported as unavailable
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable" if not self.ok else "no samples"}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step_sample(heads, q, k, v, lengths, meta, prepacked):
+    """One oracle decode step on the sampled (b, h_kv) heads: pack the tail
+    group, decode the head, attend its query heads.  Returns bytes counted
+    with the same accounting as the GPU step."""
+    import oracle as O
+    grp = meta["H_q"] // meta["H_kv"]
+    bits, g, d = meta["bits"], meta["group"], meta["D"]
+    nbytes = 0
+    for (b, h) in heads:
+        n = int(lengths[b])
+        t0 = (n - 1) // g * g
+        pk_tail = O.pack_k(k[b, h, t0:n], bits, g)
+        pv_tail = O.pack_v(v[b, h, t0:n], bits, g)
+        pk, pv = prepacked[(b, h)]
+        kh, vh = O.unpack_matrix(pk), O.unpack_matrix(pv)
+        _ = (pk_tail, pv_tail)
+        O.attend_gqa_heads(q[b, h * grp:(h + 1) * grp, 0], kh, vh, n, 1.0)
+        nbytes += attend_bytes(1, grp, 1, d, [n], bits, g) + append_bytes(1, 1, d, n - t0, bits, g)
+    return nbytes
+
+
+def cpu_oracle_rate(q, k, v, lengths, meta, n_heads: int, repeats: int = 1):
+    import oracle as O
+    rng = np.random.default_rng(123)
+    all_heads = [(b, h) for b in range(meta["B"]) for h in range(meta["H_kv"])]
+    idx = rng.choice(len(all_heads), size=min(n_heads, len(all_heads)), replace=False)
+    heads = [all_heads[i] for i in sorted(idx)]
+    pre = {(b, h): (O.pack_k(k[b, h], meta["bits"], meta["group"]),
+                    O.pack_v(v[b, h], meta["bits"], meta["group"])) for (b, h) in heads}
+    times, nbytes = [], 0
+    oracle_step_sample(heads[:1], q, k, v, lengths, meta, pre)   # warm
+    for _ in range(repeats):
+        t = time.perf_counter()
+        nbytes = oracle_step_sample(heads, q, k, v, lengths, meta, pre)
+        times.append(time.perf_counter() - t)
+    return nbytes, times, heads
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_kvq(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sm_b200 as K
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    q_np, k_np, v_np, lens_np, meta = W.gqa_case(WORKLOAD, SEED + rank)
+    q_np = torch.from_numpy(q_np).to(torch.bfloat16).float().numpy()
+    B, H_q, H_kv, D, N = meta["B"], meta["H_q"], meta["H_kv"], meta["D"], meta["N"]
+    bits, g = meta["bits"], meta["group"]
+    t0 = (N - 1) // g * g                       # tail group start (the new token is N-1)
+
+    caches = []
+    kd = torch.from_numpy(k_np).to(dev)
+    vd = torch.from_numpy(v_np).to(dev)
+    for _ in range(2):
+        c = K.PackedCache(B, H_kv, N, D, bits, g, dev)
+        K.pack(kd, vd, c)
+        caches.append(c)
+    win_k = kd[:, :, t0:N].contiguous()
+    win_v = vd[:, :, t0:N].contiguous()
+    del kd, vd
+    qd = torch.from_numpy(q_np).to(dev).to(torch.bfloat16)
+    lens = torch.from_numpy(lens_np).to(dev)
+    out = torch.empty_like(qd)
+    ws_need = K.workspace_size(caches[0], H_q, 1)
+    ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    K.check(dev)
+
+    def step(i):
+        c = caches[i & 1]
+        K.pack(win_k, win_v, c, t0=t0)
+        K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
+
+    stream = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # kernel-only timed region; attend sub-intervals for the roofline
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = K.launch_count()
+    with sampler:
+        start.record(stream)
+        for i in range(args.steps):
+            c = caches[i & 1]
+            K.pack(win_k, win_v, c, t0=t0)
+            ev[i][0].record(stream)
+            K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    launches = K.launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    K.check(dev)
+    ms = start.elapsed_time(end)
+    attend_ms = [a.elapsed_time(b) for a, b in ev]
+
+    # end-to-end through the public API with pinned host buffers
+    q_host = torch.from_numpy(q_np).to(torch.bfloat16).pin_memory()
+    kv_host_k = win_k[:, :, -1:].cpu().pin_memory()
+    kv_host_v = win_v[:, :, -1:].cpu().pin_memory()
+    o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(max(1, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e_start.record(stream)
+    for i in range(args.steps):
+        c = caches[i & 1]
+        qd.copy_(q_host, non_blocking=True)
+        win_k[:, :, -1:].copy_(kv_host_k, non_blocking=True)
+        win_v[:, :, -1:].copy_(kv_host_v, non_blocking=True)
+        K.pack(win_k, win_v, c, t0=t0)
+        K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
+        o_host.copy_(out, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end)
+    h2d = q_host.numel() * 2 + (kv_host_k.numel() + kv_host_v.numel()) * 4
+    d2h = o_host.numel() * 2
+
+    step_bytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g) + append_bytes(B, H_kv, D, N - t0, bits, g)
+    abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g)
+    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max = float(t[0]), float(t[1])
+
+    res = None
+    if rank == 0:
+        per_step_ms = ms_max / args.steps
+        value = world * step_bytes / (per_step_ms * 1e-3) / 1e9
+        e2e_value = world * step_bytes / (e2e_max / args.steps * 1e-3) / 1e9
+        att_ms = statistics.mean(attend_ms)
+        achieved = abytes / (att_ms * 1e-3) / 1e9
+        peak, peak_kind = measured_peaks()
+        kname = K.kernel_name(caches[0], H_q, 1)
+        src = os.path.join(ROOT, "sm_b200", "csrc",
+                           "attend_decode.cu" if kname.startswith("decode") else "attend_generic.cu")
+        res = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 6),
+            "us_per_step": round(per_step_ms * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "storage": "u4 codes + f32 scales (group 32), bf16 Q/O",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "H_q": H_q, "H_kv": H_kv, "d_h": D,
+                       "context": N, "bits": bits, "group": g, "lq": 1,
+                       "step": "append (re-pack tail K group + its V rows) + attend",
+                       "l2": "inputs larger than L2: 2 packed caches of 168 MB used in turn",
+                       "parallelism": f"independent batch per GPU x{world}",
+                       "attend_kernel": kname, "step_bytes": step_bytes},
+            "pct_of_8tbs": round(100 * value / world / 8000.0, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_source": f"hbm_gbs of {peak_kind}",
+                         "kernel": f"kvq_attend ({kname})", "attend_us": round(att_ms * 1e3, 3),
+                         "algorithmic_bytes_per_launch": abytes,
+                         "traffic": recorded_traffic(src)},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_max / args.steps * 1e3, 3)},
+            "gpu_launches": int(launches),
+            "clocks": sampler.summary(),
+            "impl": "kvq",
+        }
+    return res, (q_np, k_np, v_np, lens_np, meta)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=64,
+                    help="(b, h_kv) heads in the oracle's timed sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        q, k, v, lens, meta = W.gqa_case(WORKLOAD, SEED)
+        import torch
+        q = torch.from_numpy(q).to(torch.bfloat16).float().numpy()
+        per_step = max(4, args.cpu_heads // 4)
+        total, times = 0, []
+        for _ in range(args.warmup):
+            cpu_oracle_rate(q, k, v, lens, meta, per_step)
+        for _ in range(args.steps):
+            nb, ts, heads = cpu_oracle_rate(q, k, v, lens, meta, per_step)
+            total += nb
+            times.append(sum(ts))
+        value = total / sum(times) / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * sum(times) / len(times), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": meta["B"], "H_q": meta["H_q"],
+                       "H_kv": meta["H_kv"], "d_h": meta["D"], "context": meta["N"],
+                       "bits": meta["bits"], "group": meta["group"], "lq": 1},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"{per_step} of {meta['B'] * meta['H_kv']} (b, h_kv) heads per step"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res, data = run_kvq(args, rank, world, local_rank)
+    if rank == 0 and not args.no_cpu_baseline:
+        q, k, v, lens, meta = data
+        nb, ts, heads = cpu_oracle_rate(q, k, v, lens, meta, args.cpu_heads, repeats=3)
+        rate = nb / statistics.median(ts) / 1e9
+        res["cpu_baseline"] = {"value": round(rate, 4), "unit": "GB/s", "cores": blas_threads(),
+                               "kind": "oracle",
+                               "sample": f"{len(heads)} of {meta['B'] * meta['H_kv']} (b, h_kv) heads, "
+                                         f"median of 3 passes ({statistics.median(ts):.2f} s each)"}
+    if rank == 0:
+        print(json.dumps(res))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,166 @@
+/*
+ * kvq.h -- C ABI of the packed-KV attention library (libkvq.so, sm_100a).
+ *
+ * What it computes
+ * ----------------
+ * kvq_pack    Symmetric group quantization of K and V into a packed cache
+ *             ("KV分组打包：4-bit到底省了多少？", huhohoo.com/docs/llm/kv-packed-groups,
+ *             sections "一个字节里到底装了什么" and "为什么分组要同时看方向与长度"):
+ *             4-bit codes in [-7, 7] stored +7 two per byte (even code in the low
+ *             nibble), or 8-bit codes in [-127, 127] stored +127; one float32
+ *             scale = max|x| / 7 (or / 127) per group, 1 for an all-zero group;
+ *             K grouped along tokens within each channel, V along features within
+ *             each token; short groups zero-padded.  Rounding is to nearest, ties
+ *             to even; divisions are IEEE float32.
+ * kvq_attend  softmax(scale * Q K^T) V over the decoded cache, computed block
+ *             by block with the running max m, exponential sum z and weighted sum
+ *             u ("Block KV decoding: less workspace, more time",
+ *             huhohoo.com/en/docs/llm/kv-block-decode-cost, section "Do not
+ *             average independently normalized blocks"), so no decoded K/V and no
+ *             score matrix is ever written to memory.  Grouped-query attention:
+ *             query head h reads KV head h / (H_q / H_kv) ("给长前缀列一张有单位的
+ *             资源账本", section "GQA改变共享接口").  Keys at or beyond a sequence's
+ *             length take part in neither the max nor the sum (same page, section
+ *             "FlashAttention为什么不必保存整张热图").  Non-causal: every query row
+ *             reads every valid key.
+ *
+ * Conventions
+ * -----------
+ * - The library allocates nothing.  Every buffer is caller-owned device memory
+ *   unless a parameter says "host".  Calls are asynchronous on `stream` (a
+ *   cudaStream_t passed as void*; NULL is the legacy default stream).
+ * - Argument errors are found on the host before any launch and returned
+ *   synchronously; nothing is launched then.  Errors found by a kernel (a
+ *   length of 0 or beyond capacity, a bounded wait that ran out) are recorded
+ *   in a device error word and returned by kvq_check().
+ * - All tensors are dense, row-major, in the shapes stated.
+ * - Thread safety: calls on different streams may overlap; the device error
+ *   word is shared by every call on a device.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_ARG = 1,          /* bad bits/group/shape/dtype, H_q % H_kv != 0, NULL pointer */
+  KVQ_ERR_LENGTH = 2,       /* a sequence length <= 0 or > N_cap (device-detected: kvq_check) */
+  KVQ_ERR_ALIGN = 3,        /* a cache array or workspace not 16-byte aligned */
+  KVQ_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than kvq_workspace_size() */
+  KVQ_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute query) */
+  KVQ_ERR_DEVICE = 6,       /* a kernel recorded an internal inconsistency */
+  KVQ_ERR_TIMEOUT = 7,      /* a bounded wait inside a kernel ran out */
+  KVQ_ERR_UNSUPPORTED = 8   /* valid arguments outside what this build implements */
+} kvq_status;
+
+typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+/*
+ * A packed cache: four caller-owned device arrays plus the logical shape.
+ *   bits   4 or 8;  group  g, even, >= 2.
+ *   B sequences, H_kv KV heads, N_cap token capacity (shared by all
+ *   sequences), D features per head.  Let Np = ceil(N_cap/g)*g and
+ *   Dp = ceil(D/g)*g.  Per (b, h) matrix, stacked in (b, h) order:
+ *   k_codes   Np*D*bits/8 bytes: the row-major Np x D biased code matrix,
+ *             4-bit codes paired over its flattened order (a byte may
+ *             straddle two tokens when D is odd).
+ *   k_scales  (Np/g) x D float32: scale of channel d over tokens
+ *             [j*g, (j+1)*g).
+ *   v_codes   N_cap*Dp*bits/8 bytes: the row-major N_cap x Dp code matrix.
+ *   v_scales  N_cap x (Dp/g) float32: scale of token t over features
+ *             [j*g, (j+1)*g).
+ * For one (b, h) with N_cap = N these are exactly the arrays the pages
+ * store for an N x D matrix (codes, float32 scales; the int32 shape pair is
+ * the struct's N_cap/D).
+ */
+typedef struct {
+  int32_t bits, group;
+  int32_t B, H_kv, N_cap, D;
+  uint8_t* k_codes;
+  float* k_scales;
+  uint8_t* v_codes;
+  float* v_scales;
+} kvq_cache;
+
+/* Byte sizes of the four cache arrays (host).  sizes[0..3] = k_codes,
+ * k_scales, v_codes, v_scales.  Returns KVQ_ERR_ARG for an invalid shape. */
+KVQ_API kvq_status kvq_cache_sizes(int32_t bits, int32_t group, int32_t B, int32_t H_kv,
+                           int32_t N_cap, int32_t D, size_t sizes[4]);
+
+/*
+ * Quantize and pack tokens [t0, t1) of every (b, h) into the cache.
+ *   K, V     device, [B, H_kv, t1 - t0, D] in `in_dtype` (KVQ_F32 or
+ *            KVQ_BF16; bf16 is widened exactly to float32 first).
+ *   t0       multiple of g (K groups span g tokens, so a K group is only
+ *            ever packed whole); 0 <= t0 < t1 <= N_cap.
+ * A K group that ends beyond t1 is packed as if the tokens from t1 to the
+ * group's end were zero: re-packing from the group start once more tokens
+ * exist gives exactly the bytes a whole-cache pack gives.  Writes the
+ * k_codes/k_scales of groups [t0/g, ceil(t1/g)) and the v_codes/v_scales of
+ * tokens [t0, t1); nothing else.
+ * Errors: KVQ_ERR_ARG (shape/range/dtype/NULL), KVQ_ERR_CUDA (launch).
+ */
+KVQ_API kvq_status kvq_pack(const void* K, const void* V, kvq_dtype in_dtype, int32_t t0, int32_t t1,
+                    const kvq_cache* cache, void* stream);
+
+/*
+ * Attention of Q over the packed cache.
+ *   Q        device, [B, H_q, Lq, D] in q_dtype (KVQ_F32 or KVQ_BF16).
+ *   lengths  device int32 [B]: valid keys of each sequence, 1..N_cap.
+ *   H_q      multiple of cache->H_kv.   Lq >= 1 query rows per sequence.
+ *   scale    multiplies Q K^T before the softmax (1/sqrt(D) for unscaled Q,
+ *            1 when Q already carries it).
+ *   O        device, [B, H_q, Lq, D] in q_dtype.
+ *   workspace, ws_bytes   device scratch for split partials, at least
+ *            kvq_workspace_size(...) bytes, 16-byte aligned.  Its contents
+ *            on entry do not matter; it must not be shared by calls that may
+ *            run at the same time.
+ *   splits   how many CTAs share the concatenated (b, h, token-block) list;
+ *            0 = automatic (a multiple of the SM count).  Any value gives the
+ *            same result up to float rounding order.
+ * A length outside 1..N_cap is recorded for kvq_check (KVQ_ERR_LENGTH); the
+ * rows of that sequence are then written as zeros.
+ * Errors: KVQ_ERR_ARG, KVQ_ERR_ALIGN, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA,
+ * KVQ_ERR_UNSUPPORTED (D > 256).
+ */
+KVQ_API kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                      const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
+                      void* workspace, size_t ws_bytes, int32_t splits, void* stream);
+
+/* Workspace bytes kvq_attend needs for these arguments on the current
+ * device (host).  Returns 0 for invalid arguments. */
+KVQ_API size_t kvq_workspace_size(const kvq_cache* cache, int32_t H_q, int32_t Lq, int32_t splits);
+
+/* Wait for `stream`, then return and clear the device error word of the
+ * current device: KVQ_OK, KVQ_ERR_LENGTH, KVQ_ERR_TIMEOUT or
+ * KVQ_ERR_DEVICE (KVQ_ERR_CUDA if the wait itself failed). */
+KVQ_API kvq_status kvq_check(void* stream);
+
+/* Static text for a status code. */
+KVQ_API const char* kvq_strerror(kvq_status status);
+
+/* Number of kernels this library has launched in this process so far (host
+ * counter, all devices).  Used to count launches inside a timed region. */
+KVQ_API uint64_t kvq_launch_count(void);
+
+/* Name of the attention kernel kvq_attend would run for these arguments
+ * ("decode_gqa4_d128", "generic", ...), for logs and tests. */
+KVQ_API const char* kvq_attend_kernel_name(const kvq_cache* cache, int32_t H_q, int32_t Lq);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,226 @@
+"""sm_b200 -- packed-KV online-softmax attention on B200 (sm_100a).
+
+A thin ctypes binding over ``libkvq.so`` (the C ABI in ``include/kvq.h``).
+It only marshals arguments: torch tensors supply device pointers, the current
+CUDA stream and device memory; every step of quantize/pack and attention runs
+in the library's kernels.  If ``libkvq.so`` is missing the import fails: there
+is no fallback of any kind.
+
+    cache = sm_b200.PackedCache(B, H_kv, N_cap, D, bits=4, group=32)
+    sm_b200.pack(K, V, cache)                     # K, V [B, H_kv, T, D] fp32/bf16
+    O = sm_b200.attend(Q, cache, lengths, scale)  # Q [B, H_q, Lq, D] fp32/bf16
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "KVQError", "PackedCache", "pack", "attend", "workspace_size", "check",
+    "launch_count", "kernel_name", "cache_sizes", "lib", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
+
+KVQ_F32, KVQ_BF16 = 0, 1
+STATUS = {
+    0: "KVQ_OK", 1: "KVQ_ERR_ARG", 2: "KVQ_ERR_LENGTH", 3: "KVQ_ERR_ALIGN",
+    4: "KVQ_ERR_WORKSPACE", 5: "KVQ_ERR_CUDA", 6: "KVQ_ERR_DEVICE", 7: "KVQ_ERR_TIMEOUT",
+    8: "KVQ_ERR_UNSUPPORTED",
+}
+
+
+class KVQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        self.name = STATUS.get(self.status, str(status))
+        super().__init__(f"{where}: {self.name} ({lib.kvq_strerror(self.status).decode()})")
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [
+        ("bits", ctypes.c_int32), ("group", ctypes.c_int32),
+        ("B", ctypes.c_int32), ("H_kv", ctypes.c_int32),
+        ("N_cap", ctypes.c_int32), ("D", ctypes.c_int32),
+        ("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+        ("v_codes", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkvq.so not built: run `python -m sm_b200.build` ({LIB_PATH})")
+    L = ctypes.CDLL(LIB_PATH)
+    i32, vp, sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+    L.kvq_cache_sizes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]
+    L.kvq_cache_sizes.restype = ctypes.c_int
+    L.kvq_pack.argtypes = [vp, vp, ctypes.c_int, i32, i32, ctypes.POINTER(_Cache), vp]
+    L.kvq_pack.restype = ctypes.c_int
+    L.kvq_attend.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, i32, i32,
+                             ctypes.c_float, vp, vp, sz, i32, vp]
+    L.kvq_attend.restype = ctypes.c_int
+    L.kvq_workspace_size.argtypes = [ctypes.POINTER(_Cache), i32, i32, i32]
+    L.kvq_workspace_size.restype = sz
+    L.kvq_check.argtypes = [vp]
+    L.kvq_check.restype = ctypes.c_int
+    L.kvq_strerror.argtypes = [ctypes.c_int]
+    L.kvq_strerror.restype = ctypes.c_char_p
+    L.kvq_launch_count.argtypes = []
+    L.kvq_launch_count.restype = ctypes.c_uint64
+    L.kvq_attend_kernel_name.argtypes = [ctypes.POINTER(_Cache), i32, i32]
+    L.kvq_attend_kernel_name.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KVQ_F32
+    if t.dtype == torch.bfloat16:
+        return KVQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: float32 or bfloat16")
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ok(status: int, where: str) -> None:
+    if status != 0:
+        raise KVQError(status, where)
+
+
+def cache_sizes(B: int, H_kv: int, N_cap: int, D: int, bits: int = 4, group: int = 32):
+    """Byte sizes of (k_codes, k_scales, v_codes, v_scales)."""
+    out = (ctypes.c_size_t * 4)()
+    _ok(lib.kvq_cache_sizes(bits, group, B, H_kv, N_cap, D, out), "kvq_cache_sizes")
+    return tuple(int(v) for v in out)
+
+
+class PackedCache:
+    """Device memory of one packed cache, allocated through torch.
+
+    k_codes / v_codes are uint8, k_scales / v_scales float32, each flat and
+    laid out as ``include/kvq.h`` describes."""
+
+    def __init__(self, B: int, H_kv: int, N_cap: int, D: int, bits: int = 4, group: int = 32,
+                 device="cuda"):
+        self.B, self.H_kv, self.N_cap, self.D = int(B), int(H_kv), int(N_cap), int(D)
+        self.bits, self.group = int(bits), int(group)
+        kc, ks, vc, vs = cache_sizes(B, H_kv, N_cap, D, bits, group)
+        dev = torch.device(device)
+        self.k_codes = torch.zeros(kc, dtype=torch.uint8, device=dev)
+        self.k_scales = torch.zeros(ks // 4, dtype=torch.float32, device=dev)
+        self.v_codes = torch.zeros(vc, dtype=torch.uint8, device=dev)
+        self.v_scales = torch.zeros(vs // 4, dtype=torch.float32, device=dev)
+        self.device = dev
+
+    @property
+    def Np(self) -> int:
+        return -(-self.N_cap // self.group) * self.group
+
+    @property
+    def Dp(self) -> int:
+        return -(-self.D // self.group) * self.group
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.k_codes, self.k_scales, self.v_codes, self.v_scales))
+
+    def struct(self) -> _Cache:
+        return _Cache(self.bits, self.group, self.B, self.H_kv, self.N_cap, self.D,
+                      self.k_codes.data_ptr(), self.k_scales.data_ptr(),
+                      self.v_codes.data_ptr(), self.v_scales.data_ptr())
+
+    # per-(b, h) views, for tests and inspection
+    def head_k_codes(self, b: int, h: int) -> torch.Tensor:
+        n = self.k_codes.numel() // (self.B * self.H_kv)
+        i = b * self.H_kv + h
+        return self.k_codes[i * n:(i + 1) * n]
+
+    def head_v_codes(self, b: int, h: int) -> torch.Tensor:
+        n = self.v_codes.numel() // (self.B * self.H_kv)
+        i = b * self.H_kv + h
+        return self.v_codes[i * n:(i + 1) * n]
+
+    def head_k_scales(self, b: int, h: int) -> torch.Tensor:
+        return self.k_scales.view(self.B, self.H_kv, self.Np // self.group, self.D)[b, h]
+
+    def head_v_scales(self, b: int, h: int) -> torch.Tensor:
+        return self.v_scales.view(self.B, self.H_kv, self.N_cap, self.Dp // self.group)[b, h]
+
+
+def _check_cuda(t: torch.Tensor, name: str, dev: torch.device) -> None:
+    if not t.is_cuda or t.device != dev:
+        raise ValueError(f"{name} must be on {dev}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def pack(K: torch.Tensor, V: torch.Tensor, cache: PackedCache, t0: int = 0) -> None:
+    """Quantize and pack K, V [B, H_kv, T, D] into cache tokens [t0, t0 + T)."""
+    _check_cuda(K, "K", cache.device)
+    _check_cuda(V, "V", cache.device)
+    if K.shape != V.shape or K.dtype != V.dtype or K.dim() != 4:
+        raise ValueError("K and V must be [B, H_kv, T, D] of one dtype")
+    B, H, T, D = K.shape
+    if (B, H, D) != (cache.B, cache.H_kv, cache.D):
+        raise ValueError("K/V shape does not match the cache")
+    c = cache.struct()
+    _ok(lib.kvq_pack(K.data_ptr(), V.data_ptr(), _dtype_code(K), int(t0), int(t0 + T),
+                     ctypes.byref(c), _stream(cache.device)), "kvq_pack")
+
+
+def workspace_size(cache: PackedCache, H_q: int, Lq: int, splits: int = 0) -> int:
+    c = cache.struct()
+    return int(lib.kvq_workspace_size(ctypes.byref(c), int(H_q), int(Lq), int(splits)))
+
+
+def kernel_name(cache: PackedCache, H_q: int, Lq: int) -> str:
+    c = cache.struct()
+    return lib.kvq_attend_kernel_name(ctypes.byref(c), int(H_q), int(Lq)).decode()
+
+
+def attend(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, scale: float,
+           out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+           splits: int = 0) -> torch.Tensor:
+    """O = softmax(scale * Q K^T) V over the packed cache, per sequence up to
+    its length.  Q [B, H_q, Lq, D] fp32/bf16; lengths int32 [B] on the device;
+    returns O like Q (written into ``out`` if given)."""
+    _check_cuda(Q, "Q", cache.device)
+    _check_cuda(lengths, "lengths", cache.device)
+    if lengths.dtype != torch.int32 or lengths.numel() != cache.B:
+        raise ValueError("lengths must be int32 [B]")
+    if Q.dim() != 4 or Q.shape[0] != cache.B or Q.shape[3] != cache.D:
+        raise ValueError("Q must be [B, H_q, Lq, D]")
+    H_q, Lq = int(Q.shape[1]), int(Q.shape[2])
+    if out is None:
+        out = torch.empty_like(Q)
+    else:
+        _check_cuda(out, "out", cache.device)
+        if out.shape != Q.shape or out.dtype != Q.dtype:
+            raise ValueError("out must match Q")
+    need = workspace_size(cache, H_q, Lq, splits)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=cache.device)
+    c = cache.struct()
+    _ok(lib.kvq_attend(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(), H_q, Lq,
+                       float(scale), out.data_ptr(), workspace.data_ptr(),
+                       workspace.numel() * workspace.element_size(), int(splits),
+                       _stream(cache.device)), "kvq_attend")
+    return out
+
+
+def check(device=None) -> None:
+    """Wait for the current stream and raise if a kernel recorded an error."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _ok(lib.kvq_check(_stream(dev)), "kvq_check")
+
+
+def launch_count() -> int:
+    return int(lib.kvq_launch_count())

@@ -1,0 +1,138 @@
+// Internal declarations shared by the CUDA sources of libkvq.so.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+// ---------------------------------------------------------------------------
+// device error word (one per device, per loaded library)
+// ---------------------------------------------------------------------------
+// Device address of the error word of the current device (host; cached per
+// device).  Kernels receive it as a parameter and record the first error.
+unsigned int* error_word();
+
+__device__ __forceinline__ void record_error(unsigned int* err, kvq_status s) {
+  atomicCAS(err, 0u, static_cast<unsigned int>(s));
+}
+
+// host launch counter
+void count_launch(int n = 1);
+
+// SM count of the current device (cached per device)
+int sm_count();
+
+// ---------------------------------------------------------------------------
+// cache geometry
+// ---------------------------------------------------------------------------
+struct Geometry {
+  int bits, group, B, H_kv, N_cap, D;
+  int Np, Dp;                      // padded token / feature counts
+  size_t k_codes_head, k_scales_head, v_codes_head, v_scales_head;  // per (b,h), in elements
+};
+
+bool make_geometry(const kvq_cache* c, Geometry* g);
+
+// ---------------------------------------------------------------------------
+// dtype helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float load_as_f32(const void* p, size_t i, int dtype) {
+  if (dtype == KVQ_F32) return static_cast<const float*>(p)[i];
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+__device__ __forceinline__ void store_from_f32(void* p, size_t i, float v, int dtype) {
+  if (dtype == KVQ_F32) static_cast<float*>(p)[i] = v;
+  else static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+}
+
+// ---------------------------------------------------------------------------
+// work plan over the concatenated (b, h, block) list
+//
+// Blocks of BT tokens, ordered b-major, then h, then block index.  CTA c of
+// `ctas` takes the contiguous global blocks [c*P, min((c+1)*P, T)), with
+// P = ceil(T / ctas).  Whenever the CTA leaves a (b, h) it has not covered
+// whole, it writes a partial (m, z, u) into slot (c + bh): along the monotone
+// walk of (c, bh) pairs that sum is strictly increasing, so slots are unique
+// and fewer than ctas + B*H_kv.
+// ---------------------------------------------------------------------------
+struct PlanArgs {
+  const int32_t* lengths;
+  int B, H_kv, N_cap, BT, ctas;
+};
+
+// per-sequence block count with the length clamped to [0, N_cap]
+__device__ __forceinline__ int seq_blocks(int len, int n_cap, int bt) {
+  len = len < 0 ? 0 : (len > n_cap ? n_cap : len);
+  return (len + bt - 1) / bt;
+}
+
+// Merge partial states of a split (b, h) and write the output rows.
+struct MergeArgs {
+  const float* partials;           // [slots][R_pad][D + 2] : m, z, u[D]
+  const int32_t* lengths;
+  void* O;
+  int o_dtype;
+  int B, H_kv, N_cap, BT, ctas;
+  int R, R_pad, D;                 // rows per (b,h) and the padded row count of a slot
+  int G, Lq;                       // query heads per KV head, rows per query head
+};
+kvq_status launch_merge(const MergeArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// kernels' host launchers
+// ---------------------------------------------------------------------------
+struct PackArgs {
+  const void* K;
+  const void* V;
+  int in_dtype;
+  int t0, t1;
+  Geometry g;
+  uint8_t* k_codes;
+  float* k_scales;
+  uint8_t* v_codes;
+  float* v_scales;
+};
+kvq_status launch_pack(const PackArgs& a, cudaStream_t s);
+
+struct AttendArgs {
+  const void* Q;
+  int q_dtype;
+  Geometry g;
+  const uint8_t* k_codes;
+  const float* k_scales;
+  const uint8_t* v_codes;
+  const float* v_scales;
+  const int32_t* lengths;
+  int H_q, Lq;
+  float scale;
+  void* O;
+  void* workspace;
+  size_t ws_bytes;
+  int splits;
+};
+
+// One implementation of kvq_attend: how much workspace it needs and how to
+// launch it.  `applies` says whether it handles these arguments.
+struct AttendImpl {
+  const char* name;
+  bool (*applies)(const AttendArgs&);
+  size_t (*workspace)(const AttendArgs&);
+  kvq_status (*launch)(const AttendArgs&, cudaStream_t);
+};
+
+const AttendImpl& generic_attend_impl();
+const AttendImpl* decode_attend_impl();     // tuned decode; nullptr if not built
+const AttendImpl* chunk_attend_impl();      // tensor-core chunk; nullptr if not built
+
+// Partial-slot bound shared by every split implementation.
+inline size_t partial_slots(int ctas, int B, int H_kv) {
+  return static_cast<size_t>(ctas) + static_cast<size_t>(B) * static_cast<size_t>(H_kv);
+}
+
+}  // namespace kvq

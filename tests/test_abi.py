@@ -1,0 +1,118 @@
+"""CPU tests of the C ABI: the library loads, exports every function
+include/kvq.h declares, sizes its arrays like the oracle's, and rejects bad
+arguments on the host before any launch (fake pointers are never touched)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle as O
+import sm_b200 as K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    return re.findall(r"KVQ_API\s+[\w\s\*]+?\b(kvq_\w+)\s*\(", text)
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert len(names) >= 8
+    out = subprocess.run(["nm", "-D", "--defined-only", K.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(K.lib, n)
+    # nothing but the C ABI leaks out
+    assert {e for e in exported if e.startswith("kvq")} == set(names)
+
+
+def test_strerror_covers_every_status():
+    for code, name in K.STATUS.items():
+        text = K.lib.kvq_strerror(code).decode()
+        assert text and text != "unknown status", name
+    assert K.lib.kvq_strerror(99).decode() == "unknown status"
+
+
+@pytest.mark.parametrize("bits,group,n,d", [(4, 32, 128, 32), (4, 8, 35, 13), (8, 8, 35, 13),
+                                            (8, 32, 512, 32), (4, 32, 4096, 128)])
+def test_cache_sizes_match_oracle_arrays(bits, group, n, d):
+    x = np.zeros((n, d), np.float32)
+    pk, pv = O.pack_k(x, bits, group), O.pack_v(x, bits, group)
+    heads = 3 * 2
+    kc, ks, vc, vs = K.cache_sizes(3, 2, n, d, bits, group)
+    assert kc == heads * pk.codes.nbytes
+    assert ks == heads * pk.scales.nbytes
+    assert vc == heads * pv.codes.nbytes
+    assert vs == heads * pv.scales.nbytes
+
+
+def _cache(bits=4, group=32, B=2, H=2, N=64, D=32, ptr=0x10000):
+    return K._Cache(bits, group, B, H, N, D, ptr, ptr + 0x100000, ptr + 0x200000, ptr + 0x300000)
+
+
+@pytest.mark.parametrize("bad", [dict(bits=5), dict(bits=2), dict(group=7), dict(group=0),
+                                 dict(B=0), dict(H=0), dict(N=0), dict(D=0)])
+def test_bad_cache_rejected(bad):
+    c = _cache(**bad)
+    st = K.lib.kvq_pack(0x1000, 0x2000, K.KVQ_F32, 0, 8, ctypes.byref(c), None)
+    assert st == 1
+    st = K.lib.kvq_attend(0x1000, K.KVQ_BF16, ctypes.byref(c), 0x3000, 4, 1, 1.0, 0x4000,
+                          0x5000, 1 << 30, 0, None)
+    assert st == 1
+    assert K.lib.kvq_workspace_size(ctypes.byref(c), 4, 1, 0) == 0
+
+
+def test_pack_range_rules():
+    c = _cache(group=32, N=64)
+    call = lambda t0, t1, dt=K.KVQ_F32, kp=0x1000: K.lib.kvq_pack(kp, 0x2000, dt, t0, t1,
+                                                                 ctypes.byref(c), None)
+    assert call(8, 40) == 1          # t0 not a group start
+    assert call(0, 0) == 1           # empty range
+    assert call(32, 16) == 1         # reversed
+    assert call(0, 65) == 1          # beyond capacity
+    assert call(-32, 8) == 1
+    assert call(0, 8, dt=7) == 1     # unknown dtype
+    assert call(0, 8, kp=0) == 1     # NULL input
+    assert call(0, 8, kp=0x1002) == 3  # misaligned float32 input
+
+
+def test_attend_argument_rules():
+    c = _cache()
+    ws = 1 << 30
+
+    def call(q=0x1000, dt=K.KVQ_BF16, cache=c, lens=0x3000, hq=4, lq=1, o=0x4000, w=0x5000,
+             wsb=ws, splits=0):
+        return K.lib.kvq_attend(q, dt, ctypes.byref(cache), lens, hq, lq, 1.0, o, w, wsb, splits,
+                                None)
+
+    assert call(hq=3) == 1                       # H_q not a multiple of H_kv
+    assert call(hq=0) == 1
+    assert call(lq=0) == 1
+    assert call(dt=3) == 1
+    assert call(splits=-1) == 1
+    assert call(q=0) == 1 and call(o=0) == 1 and call(lens=0) == 1
+    assert call(cache=_cache(ptr=0x10008)) == 3  # cache arrays not 16-byte aligned
+    assert call(q=0x1001) == 3                   # bf16 Q misaligned
+    assert call(lens=0x3002) == 3
+    assert call(cache=_cache(D=300)) == 8        # unsupported width
+    assert call(w=0) == 4                        # no workspace
+    assert call(wsb=16) == 4                     # too small
+    assert call(w=0x5008) == 3                   # misaligned workspace
+
+
+def test_workspace_size_grows_with_splits():
+    c = _cache(B=4, H=2, N=4096, D=128)
+    a = K.lib.kvq_workspace_size(ctypes.byref(c), 8, 1, 8)
+    b = K.lib.kvq_workspace_size(ctypes.byref(c), 8, 1, 64)
+    assert 0 < a < b

@@ -1,0 +1,227 @@
+"""GPU parity: kvq_pack bit-exact against the oracle, kvq_attend within
+2e-3 * max|V_hat| of the float64 oracle on the same decoded cache, on every
+workload shape -- the single-head grid, the 35 x 13 edge case, ragged GQA
+cases spanning several blocks and a tail, and the full-size decode,
+long-context and chunk workloads (sampled heads)."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from tests.gpu_util import (DEV, assert_head_packed_equal, bf16_values, check_rows, oracle_rows,
+                            pack_gpu, single_head_scale, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sm():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sm_b200
+    return sm_b200
+
+
+# ---------------------------------------------------------------------------
+# pack
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,group", W.FORMATS)
+def test_pack_single_head_grid(sm, bits, group):
+    for n, seed, dist in W.SINGLE_HEAD_GRID:
+        q, k, v = W.single_head(n, 32, 4, seed, dist)
+        cache = pack_gpu(sm, k[None, None], v[None, None], bits, group)
+        assert_head_packed_equal(cache, 0, 0, O.pack_k(k, bits, group), O.pack_v(v, bits, group))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("group", [8, 32])
+@pytest.mark.parametrize("in_dtype", [torch.float32, torch.bfloat16])
+def test_pack_35x13(sm, bits, group, in_dtype):
+    _, k, v = W.edge_35x13(0)
+    if in_dtype == torch.bfloat16:
+        k, v = bf16_values(k), bf16_values(v)
+    cache = pack_gpu(sm, k[None, None], v[None, None], bits, group, in_dtype)
+    assert_head_packed_equal(cache, 0, 0, O.pack_k(k, bits, group), O.pack_v(v, bits, group))
+
+
+def test_pack_all_zero_and_ties(sm):
+    z = np.zeros((1, 1, 35, 13), np.float32)
+    cache = pack_gpu(sm, z, z, 4, 8)
+    assert_head_packed_equal(cache, 0, 0, O.pack_k(z[0, 0], 4, 8), O.pack_v(z[0, 0], 4, 8))
+    ties = np.array([[0.5, 1.5, 2.5, 7.0, -0.5, -1.5, -2.5, -7.0]] * 4, np.float32)
+    cache = pack_gpu(sm, ties[None, None], ties[None, None], 4, 8)
+    assert_head_packed_equal(cache, 0, 0, O.pack_k(ties, 4, 8), O.pack_v(ties, 4, 8))
+
+
+def test_pack_append_matches_whole(sm):
+    """Packing [0, 64) then [64, 100) then re-packing the tail group from its
+    start, [96, 130), gives the bytes of a whole [0, 130) pack."""
+    rng = np.random.default_rng(4)
+    k = rng.standard_normal((2, 3, 130, 40)).astype(np.float32)
+    v = rng.standard_normal((2, 3, 130, 40)).astype(np.float32)
+    whole = pack_gpu(sm, k, v, 4, 32)
+    part = sm.PackedCache(2, 3, 130, 40, 4, 32, DEV)
+    sm.pack(to_dev(k[:, :, 0:64]), to_dev(v[:, :, 0:64]), part, t0=0)
+    sm.pack(to_dev(k[:, :, 64:100]), to_dev(v[:, :, 64:100]), part, t0=64)
+    sm.pack(to_dev(k[:, :, 96:130]), to_dev(v[:, :, 96:130]), part, t0=96)
+    for a, b in ((whole.k_codes, part.k_codes), (whole.v_codes, part.v_codes),
+                 (whole.k_scales, part.k_scales), (whole.v_scales, part.v_scales)):
+        assert torch.equal(a, b)
+    for b_ in range(2):
+        for h in range(3):
+            assert_head_packed_equal(whole, b_, h, O.pack_k(k[b_, h], 4, 32), O.pack_v(v[b_, h], 4, 32))
+
+
+# ---------------------------------------------------------------------------
+# attend: single-head grid (72 comparisons) and the 35 x 13 case
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,group", W.FORMATS)
+def test_attend_single_head_grid(sm, bits, group):
+    worst = 0.0
+    for n, seed, dist in W.SINGLE_HEAD_GRID:
+        q, k, v = W.single_head(n, 32, 4, seed, dist)
+        cache = pack_gpu(sm, k[None, None], v[None, None], bits, group)
+        lens = torch.tensor([n], dtype=torch.int32, device=DEV)
+        out = sm.attend(to_dev(q[None, None]), cache, lens, single_head_scale(32))
+        want, pk, pv, vh = oracle_rows(q, k, v, bits, group, n, single_head_scale(32))
+        worst = max(worst, check_rows(out[0, 0].cpu().numpy(), want, vh, f"{n}/{seed}/{dist}"))
+    sm.check()
+
+
+@pytest.mark.parametrize("bits,group", W.FORMATS)
+def test_attend_35x13(sm, bits, group):
+    q, k, v = W.edge_35x13(0)
+    cache = pack_gpu(sm, k[None, None], v[None, None], bits, group)
+    lens = torch.tensor([35], dtype=torch.int32, device=DEV)
+    out = sm.attend(to_dev(q[None, None]), cache, lens, single_head_scale(13))
+    want, *_, vh = oracle_rows(q, k, v, bits, group, 35, single_head_scale(13))
+    check_rows(out[0, 0].cpu().numpy(), want, vh, "35x13")
+    # also against the pages' block-7 decode-and-merge path
+    blk = O.attend_blocked_packed(q, O.pack_k(k, bits, group), O.pack_v(v, bits, group),
+                                  single_head_scale(13), 7)
+    check_rows(out[0, 0].cpu().numpy(), blk, vh, "35x13 vs block 7")
+
+
+# ---------------------------------------------------------------------------
+# attend: ragged GQA cases, split invariance, dtype, lengths
+# ---------------------------------------------------------------------------
+
+def _gqa_case(b_, hq, hkv, n_cap, d, lens, lq=1, seed=0, bits=4, group=32, outliers=False):
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((b_, hkv, n_cap, d)).astype(np.float32)
+    v = rng.standard_normal((b_, hkv, n_cap, d)).astype(np.float32)
+    if outliers:
+        k[:, :, :, ::37] *= 8
+        v[:, :, :, 5::41] *= 8
+    q = (rng.standard_normal((b_, hq, lq, d)) / math.sqrt(d)).astype(np.float32)
+    return q, k, v, np.asarray(lens, np.int32)
+
+
+def _check_gqa(sm, q, k, v, lens, bits, group, scale, q_dtype=torch.bfloat16, splits=0,
+               heads=None, out_dtype_check=True):
+    b_, hq, lq, d = q.shape
+    hkv = k.shape[1]
+    grp = hq // hkv
+    cache = pack_gpu(sm, k, v, bits, group)
+    qd = to_dev(q, q_dtype)
+    qv = qd.float().cpu().numpy()
+    out = sm.attend(qd, cache, to_dev(lens, torch.int32), scale, splits=splits)
+    sm.check()
+    assert out.dtype == q_dtype
+    o = out.float().cpu().numpy()
+    sel = heads if heads is not None else [(b, h) for b in range(b_) for h in range(hkv)]
+    for b, h in sel:
+        rows = qv[b, h * grp:(h + 1) * grp].reshape(grp * lq, d)
+        want, pk, pv, vh = oracle_rows(rows, k[b, h], v[b, h], bits, group, int(lens[b]), scale)
+        assert_head_packed_equal(cache, b, h, pk, pv)
+        got = o[b, h * grp:(h + 1) * grp].reshape(grp * lq, d)
+        check_rows(got, want, vh, f"b{b} h{h}")
+    return o
+
+
+@pytest.mark.parametrize("splits", [0, 1, 2, 7, 1000])
+def test_gqa_ragged_split_invariance(sm, splits):
+    # lengths not multiples of 32 or 128, one of a single token, capacity 300
+    q, k, v, lens = _gqa_case(3, 8, 2, 300, 128, [300, 157, 1])
+    _check_gqa(sm, q, k, v, lens, 4, 32, 1.0, splits=splits)
+
+
+@pytest.mark.parametrize("bits,group", W.FORMATS)
+def test_gqa_formats_fp32_q(sm, bits, group):
+    q, k, v, lens = _gqa_case(2, 4, 1, 200, 64, [200, 77], seed=3)
+    _check_gqa(sm, q, k, v, lens, bits, group, 1.0, q_dtype=torch.float32)
+
+
+def test_gqa_multi_query_rows(sm):
+    q, k, v, lens = _gqa_case(2, 8, 2, 260, 128, [260, 129], lq=5, seed=5, outliers=True)
+    _check_gqa(sm, q, k, v, lens, 4, 32, 1.0)
+
+
+def test_repeat_is_bit_identical(sm):
+    q, k, v, lens = _gqa_case(2, 8, 2, 300, 128, [300, 200], seed=6)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    qd, ld = to_dev(q, torch.bfloat16), to_dev(lens, torch.int32)
+    a = sm.attend(qd, cache, ld, 1.0, splits=5)
+    b = sm.attend(qd, cache, ld, 1.0, splits=5)
+    assert torch.equal(a, b)
+
+
+def test_every_output_written(sm):
+    q, k, v, lens = _gqa_case(2, 8, 2, 300, 128, [300, 33], seed=7)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+    sm.attend(to_dev(q, torch.bfloat16), cache, to_dev(lens, torch.int32), 1.0, out=out, splits=3)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_bad_lengths_reported(sm):
+    q, k, v, _ = _gqa_case(3, 4, 2, 64, 32, [64, 64, 64], seed=8)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+    lens = torch.tensor([64, 0, 64], dtype=torch.int32, device=DEV)
+    sm.attend(to_dev(q, torch.bfloat16), cache, lens, 1.0, out=out)
+    with pytest.raises(sm.KVQError) as e:
+        sm.check()
+    assert e.value.name == "KVQ_ERR_LENGTH"
+    assert torch.all(out[1] == 0)
+    assert torch.isfinite(out.float()).all()
+    sm.check()                     # the error word was cleared
+    lens = torch.tensor([64, 65, 64], dtype=torch.int32, device=DEV)
+    sm.attend(to_dev(q, torch.bfloat16), cache, lens, 1.0, out=out)
+    with pytest.raises(sm.KVQError):
+        sm.check()
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled heads
+# ---------------------------------------------------------------------------
+
+SAMPLE = [(0, 0), (5, 3), (17, 7), (31, 1)]
+
+
+def _full_case(sm, name, seed=0, bits=4, heads=SAMPLE, splits=0):
+    q, k, v, lens, meta = W.gqa_case(name, seed)
+    q = bf16_values(q)
+    _check_gqa(sm, q, k, v, lens, bits, meta["group"], 1.0, splits=splits,
+               heads=[(b % meta["B"], h) for b, h in heads])
+
+
+def test_decode_gqa_full(sm):
+    _full_case(sm, "decode_gqa")
+
+
+def test_long_context_full(sm):
+    _full_case(sm, "long_context", heads=[(0, 0), (3, 5), (7, 7), (6, 2)])
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_chunk_full(sm, bits):
+    _full_case(sm, "chunk", bits=bits, heads=[(0, 0), (1, 5), (3, 7)])
