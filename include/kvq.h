@@ -139,6 +139,37 @@ KVQ_API kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache*
                       const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
                       void* workspace, size_t ws_bytes, int32_t splits, void* stream);
 
+/*
+ * kvq_attend without a caller workspace, for callers that cannot allocate
+ * device memory when they call: code inside an engine that reserves all its
+ * device memory at start-up and allows no allocation afterwards, or a hot
+ * loop where a cudaMalloc would synchronize the device and stall other
+ * streams.  The pages have no counterpart; this is a library convenience.
+ *
+ * Same arguments and results as kvq_attend minus workspace/ws_bytes.  The
+ * split-KV scratch is a fixed array of KVQ_NOALLOC_SCRATCH_BYTES compiled
+ * into the library; every GPU that loads the library holds it until the
+ * process exits.  The function allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library call).
+ * - Limit: if kvq_workspace_size(cache, H_q, Lq, splits) exceeds
+ *   KVQ_NOALLOC_SCRATCH_BYTES the call returns KVQ_ERR_WORKSPACE and
+ *   launches nothing; use kvq_attend with your own workspace instead.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls on a device share the one array and it keeps the previous
+ *   call's contents (no state is carried from one call to the next); calls
+ *   whose kernels may overlap on the GPU race on it, so order them (one
+ *   stream, or events).
+ */
+#define KVQ_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+KVQ_API kvq_status kvq_attend_noalloc(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                      const int32_t* lengths, int32_t H_q, int32_t Lq,
+                                      float scale, void* O, int32_t splits, void* stream);
+
+/* Size in bytes of the fixed scratch array kvq_attend_noalloc uses. */
+KVQ_API size_t kvq_noalloc_scratch_bytes(void);
+
 /* Workspace bytes kvq_attend needs for these arguments on the current
  * device (host).  Returns 0 for invalid arguments. */
 KVQ_API size_t kvq_workspace_size(const kvq_cache* cache, int32_t H_q, int32_t Lq, int32_t splits);

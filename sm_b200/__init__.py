@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "KVQError", "PackedCache", "pack", "attend", "workspace_size", "check",
-    "launch_count", "kernel_name", "cache_sizes", "lib", "LIB_PATH",
+    "launch_count", "kernel_name", "cache_sizes", "lib", "LIB_PATH", "attend_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
@@ -72,6 +72,11 @@ def _load() -> ctypes.CDLL:
     L.kvq_launch_count.restype = ctypes.c_uint64
     L.kvq_attend_kernel_name.argtypes = [ctypes.POINTER(_Cache), i32, i32]
     L.kvq_attend_kernel_name.restype = ctypes.c_char_p
+    L.kvq_attend_noalloc.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, i32, i32,
+                                     ctypes.c_float, vp, i32, vp]
+    L.kvq_attend_noalloc.restype = ctypes.c_int
+    L.kvq_noalloc_scratch_bytes.argtypes = []
+    L.kvq_noalloc_scratch_bytes.restype = sz
     return L
 
 
@@ -213,6 +218,29 @@ def attend(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, scale: fl
                        float(scale), out.data_ptr(), workspace.data_ptr(),
                        workspace.numel() * workspace.element_size(), int(splits),
                        _stream(cache.device)), "kvq_attend")
+    return out
+
+
+def attend_noalloc(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, scale: float,
+                   out: torch.Tensor | None = None, splits: int = 0) -> torch.Tensor:
+    """attend() for callers that cannot allocate device memory when they call
+    (an engine that reserved all of its memory at start-up, or a loop where a
+    cudaMalloc would stall other streams): the split scratch is a fixed array
+    inside the library, shared by every call on the device, so calls that may
+    run at the same time on one device must be ordered.  ``out`` must then be
+    preallocated by the caller; this wrapper only creates it when omitted."""
+    _check_cuda(Q, "Q", cache.device)
+    _check_cuda(lengths, "lengths", cache.device)
+    if lengths.dtype != torch.int32 or lengths.numel() != cache.B:
+        raise ValueError("lengths must be int32 [B]")
+    if Q.dim() != 4 or Q.shape[0] != cache.B or Q.shape[3] != cache.D:
+        raise ValueError("Q must be [B, H_q, Lq, D]")
+    if out is None:
+        out = torch.empty_like(Q)
+    c = cache.struct()
+    _ok(lib.kvq_attend_noalloc(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(),
+                               int(Q.shape[1]), int(Q.shape[2]), float(scale), out.data_ptr(),
+                               int(splits), _stream(cache.device)), "kvq_attend_noalloc")
     return out
 
 
