@@ -7,9 +7,9 @@ context 4096 for every sequence, 4-bit codes in groups of 32 with float32
 scales, bf16 Q and O.  One step is one pass of the whole hot path for a
 decode step:
 
-  1. append -- kvq_pack re-packs the tail K group (tokens 4064..4095, where
-     the new token sits) and the V rows of those tokens from a float32
-     recent-token window, and
+  1. append -- kvq_pack re-packs the K group that holds the new token
+     (tokens 4064..4095) from a float32 recent-token window, and packs the
+     new token's V row (token 4095), and
   2. attend -- kvq_attend over the whole 4096-token packed cache.
 
 Two independent packed caches (2 x 168 MB, more than the 126 MB L2) are used
@@ -70,12 +70,14 @@ def attend_bytes(B, H_q, H_kv, D, lengths, bits=4, group=32, q_bytes=2, o_bytes=
     return total
 
 
-def append_bytes(B, H_kv, D, tokens, bits=4, group=32, in_bytes=4):
+def append_bytes(B, H_kv, D, k_tokens, v_tokens=1, bits=4, group=32, in_bytes=4):
+    """Bytes of the decode-step append: the K tail group (k_tokens float32
+    rows in, their codes and the group's scale row out) and the new V rows
+    (v_tokens float32 rows in, codes and scales out)."""
     dp = -(-D // group) * group
-    per_head = (2 * tokens * D * in_bytes                     # K, V window in
-                + tokens * D * bits // 8 + tokens * dp * bits // 8   # codes out
-                + -(-tokens // group) * D * 4 + tokens * (dp // group) * 4)  # scales out
-    return B * H_kv * per_head
+    k = k_tokens * D * in_bytes + k_tokens * D * bits // 8 + -(-k_tokens // group) * D * 4
+    v = v_tokens * D * in_bytes + v_tokens * dp * bits // 8 + v_tokens * (dp // group) * 4
+    return B * H_kv * (k + v)
 
 
 # ---------------------------------------------------------------------------
@@ -194,12 +196,13 @@ def oracle_step_sample(heads, q, k, v, lengths, meta, prepacked):
         n = int(lengths[b])
         t0 = (n - 1) // g * g
         pk_tail = O.pack_k(k[b, h, t0:n], bits, g)
-        pv_tail = O.pack_v(v[b, h, t0:n], bits, g)
+        pv_new = O.pack_v(v[b, h, n - 1:n], bits, g)
         pk, pv = prepacked[(b, h)]
         kh, vh = O.unpack_matrix(pk), O.unpack_matrix(pv)
-        _ = (pk_tail, pv_tail)
+        _ = (pk_tail, pv_new)
         O.attend_gqa_heads(q[b, h * grp:(h + 1) * grp, 0], kh, vh, n, 1.0)
-        nbytes += attend_bytes(1, grp, 1, d, [n], bits, g) + append_bytes(1, 1, d, n - t0, bits, g)
+        nbytes += (attend_bytes(1, grp, 1, d, [n], bits, g)
+                   + append_bytes(1, 1, d, n - t0, 1, bits, g))
     return nbytes
 
 
@@ -244,8 +247,8 @@ def run_kvq(args, rank, world, local_rank):
         c = K.PackedCache(B, H_kv, N, D, bits, g, dev)
         K.pack(kd, vd, c)
         caches.append(c)
-    win_k = kd[:, :, t0:N].contiguous()
-    win_v = vd[:, :, t0:N].contiguous()
+    win_k = kd[:, :, t0:N].contiguous()          # K of the tail group (recent-token window)
+    new_v = vd[:, :, N - 1:N].contiguous()       # V of the new token
     del kd, vd
     qd = torch.from_numpy(q_np).to(dev).to(torch.bfloat16)
     lens = torch.from_numpy(lens_np).to(dev)
@@ -257,44 +260,73 @@ def run_kvq(args, rank, world, local_rank):
 
     def step(i):
         c = caches[i & 1]
-        K.pack(win_k, win_v, c, t0=t0)
+        K.pack(win_k, None, c, t0=t0)
+        K.pack(None, new_v, c, t0=N - 1)
         K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
+
+    def attend_only(i):
+        K.attend(qd, caches[i & 1], lens, 1.0, out=out, workspace=ws)
 
     stream = torch.cuda.current_stream(dev)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
 
-    # kernel-only timed region; attend sub-intervals for the roofline
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    # The kernel-only region replays CUDA graphs of one step (append + attend
+    # on cache 0, then on cache 1), so host launch overhead does not pace it.
+    def capture(fn):
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        n0 = K.launch_count()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        torch.cuda.synchronize()
+        return g, K.launch_count() - n0
+
+    step_graphs = [capture(lambda i=i: step(i)) for i in range(2)]
+    attend_graphs = [capture(lambda i=i: attend_only(i)) for i in range(2)]
+    launches_per_step = step_graphs[0][1]
+    for i in range(args.warmup):
+        step_graphs[i & 1][0].replay()
+        attend_graphs[i & 1][0].replay()
+    torch.cuda.synchronize()
+
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    n0 = K.launch_count()
     with sampler:
         start.record(stream)
         for i in range(args.steps):
-            c = caches[i & 1]
-            K.pack(win_k, win_v, c, t0=t0)
-            ev[i][0].record(stream)
-            K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
-            ev[i][1].record(stream)
+            step_graphs[i & 1][0].replay()
         end.record(stream)
         torch.cuda.synchronize()
-    launches = K.launch_count() - n0
+    launches = launches_per_step * args.steps
     if world > 1:
         dist.barrier()
     K.check(dev)
     ms = start.elapsed_time(end)
-    attend_ms = [a.elapsed_time(b) for a, b in ev]
 
-    # end-to-end through the public API with pinned host buffers
+    # the attend kernel alone, same caches in turn, for the roofline
+    a_start, a_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_start.record(stream)
+    for i in range(args.steps):
+        attend_graphs[i & 1][0].replay()
+    a_end.record(stream)
+    torch.cuda.synchronize()
+    attend_ms = [a_start.elapsed_time(a_end) / args.steps]
+
+    # end-to-end through the public API (direct calls, no graphs) with the
+    # step's inputs copied from pinned host buffers and the output read back
     q_host = torch.from_numpy(q_np).to(torch.bfloat16).pin_memory()
     kv_host_k = win_k[:, :, -1:].cpu().pin_memory()
-    kv_host_v = win_v[:, :, -1:].cpu().pin_memory()
+    kv_host_v = new_v.cpu().pin_memory()
     o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for i in range(max(1, args.warmup)):
@@ -307,8 +339,9 @@ def run_kvq(args, rank, world, local_rank):
         c = caches[i & 1]
         qd.copy_(q_host, non_blocking=True)
         win_k[:, :, -1:].copy_(kv_host_k, non_blocking=True)
-        win_v[:, :, -1:].copy_(kv_host_v, non_blocking=True)
-        K.pack(win_k, win_v, c, t0=t0)
+        new_v.copy_(kv_host_v, non_blocking=True)
+        K.pack(win_k, None, c, t0=t0)
+        K.pack(None, new_v, c, t0=N - 1)
         K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
         o_host.copy_(out, non_blocking=True)
     e_end.record(stream)
@@ -317,7 +350,7 @@ def run_kvq(args, rank, world, local_rank):
     h2d = q_host.numel() * 2 + (kv_host_k.numel() + kv_host_v.numel()) * 4
     d2h = o_host.numel() * 2
 
-    step_bytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g) + append_bytes(B, H_kv, D, N - t0, bits, g)
+    step_bytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g) + append_bytes(B, H_kv, D, N - t0, 1, bits, g)
     abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g)
     t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -344,15 +377,17 @@ def run_kvq(args, rank, world, local_rank):
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "B": B, "H_q": H_q, "H_kv": H_kv, "d_h": D,
                        "context": N, "bits": bits, "group": g, "lq": 1,
-                       "step": "append (re-pack tail K group + its V rows) + attend",
+                       "step": "append (re-pack the K group of the new token, pack its V row) + attend",
                        "l2": "inputs larger than L2: 2 packed caches of 168 MB used in turn",
                        "parallelism": f"independent batch per GPU x{world}",
-                       "attend_kernel": kname, "step_bytes": step_bytes},
+                       "attend_kernel": kname, "step_bytes": step_bytes,
+                       "launch": "CUDA graph per step (append + attend)"},
             "pct_of_8tbs": round(100 * value / world / 8000.0, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_source": f"hbm_gbs of {peak_kind}",
                          "kernel": f"kvq_attend ({kname})", "attend_us": round(att_ms * 1e3, 3),
+                         "timing": "attend-only CUDA-graph replays, same caches in turn",
                          "algorithmic_bytes_per_launch": abytes,
                          "traffic": recorded_traffic(src)},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,

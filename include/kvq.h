@@ -102,15 +102,19 @@ KVQ_API kvq_status kvq_cache_sizes(int32_t bits, int32_t group, int32_t B, int32
 /*
  * Quantize and pack tokens [t0, t1) of every (b, h) into the cache.
  *   K, V     device, [B, H_kv, t1 - t0, D] in `in_dtype` (KVQ_F32 or
- *            KVQ_BF16; bf16 is widened exactly to float32 first).
- *   t0       multiple of g (K groups span g tokens, so a K group is only
- *            ever packed whole); 0 <= t0 < t1 <= N_cap.
+ *            KVQ_BF16; bf16 is widened exactly to float32 first).  Either
+ *            may be NULL to leave that half of the cache untouched (not
+ *            both): a decode step re-packs the K group that holds the new
+ *            token and packs the new token's V row alone.
+ *   t0       with K: a multiple of g (K groups span g tokens, so a K group
+ *            is only ever packed whole); 0 <= t0 < t1 <= N_cap.
  * A K group that ends beyond t1 is packed as if the tokens from t1 to the
  * group's end were zero: re-packing from the group start once more tokens
  * exist gives exactly the bytes a whole-cache pack gives.  Writes the
  * k_codes/k_scales of groups [t0/g, ceil(t1/g)) and the v_codes/v_scales of
  * tokens [t0, t1); nothing else.
- * Errors: KVQ_ERR_ARG (shape/range/dtype/NULL), KVQ_ERR_CUDA (launch).
+ * Errors: KVQ_ERR_ARG (shape/range/dtype/NULL), KVQ_ERR_ALIGN (input not
+ * aligned to its element size), KVQ_ERR_CUDA (launch).
  */
 KVQ_API kvq_status kvq_pack(const void* K, const void* V, kvq_dtype in_dtype, int32_t t0, int32_t t1,
                     const kvq_cache* cache, void* stream);

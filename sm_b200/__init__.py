@@ -167,18 +167,25 @@ def _check_cuda(t: torch.Tensor, name: str, dev: torch.device) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
-def pack(K: torch.Tensor, V: torch.Tensor, cache: PackedCache, t0: int = 0) -> None:
-    """Quantize and pack K, V [B, H_kv, T, D] into cache tokens [t0, t0 + T)."""
-    _check_cuda(K, "K", cache.device)
-    _check_cuda(V, "V", cache.device)
-    if K.shape != V.shape or K.dtype != V.dtype or K.dim() != 4:
-        raise ValueError("K and V must be [B, H_kv, T, D] of one dtype")
-    B, H, T, D = K.shape
+def pack(K: torch.Tensor | None, V: torch.Tensor | None, cache: PackedCache, t0: int = 0) -> None:
+    """Quantize and pack K, V [B, H_kv, T, D] into cache tokens [t0, t0 + T).
+    Either may be None to pack only the other half (with K, t0 must be a
+    multiple of the group)."""
+    if K is None and V is None:
+        raise ValueError("K and V are both None")
+    ref = K if K is not None else V
+    for name, X in (("K", K), ("V", V)):
+        if X is not None:
+            _check_cuda(X, name, cache.device)
+            if X.shape != ref.shape or X.dtype != ref.dtype or X.dim() != 4:
+                raise ValueError("K and V must be [B, H_kv, T, D] of one dtype")
+    B, H, T, D = ref.shape
     if (B, H, D) != (cache.B, cache.H_kv, cache.D):
         raise ValueError("K/V shape does not match the cache")
     c = cache.struct()
-    _ok(lib.kvq_pack(K.data_ptr(), V.data_ptr(), _dtype_code(K), int(t0), int(t0 + T),
-                     ctypes.byref(c), _stream(cache.device)), "kvq_pack")
+    _ok(lib.kvq_pack(K.data_ptr() if K is not None else None,
+                     V.data_ptr() if V is not None else None, _dtype_code(ref), int(t0),
+                     int(t0 + T), ctypes.byref(c), _stream(cache.device)), "kvq_pack")
 
 
 def workspace_size(cache: PackedCache, H_q: int, Lq: int, splits: int = 0) -> int:

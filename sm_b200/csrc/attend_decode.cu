@@ -1,0 +1,714 @@
+// Tuned decode attention: D = 128, 4-bit codes, groups of 32, four query
+// heads per KV head (GQA), one query row per sequence.
+//
+// What it computes is the block rule of "Block KV decoding: less workspace,
+// more time" (huhohoo.com/en/docs/llm/kv-block-decode-cost, section "Do not
+// average independently normalized blocks") over the packed format of
+// "KV分组打包：4-bit到底省了多少？" (huhohoo.com/docs/llm/kv-packed-groups,
+// section "一个字节里到底装了什么"); each GQA group of four query heads reads its
+// KV head once ("给长前缀列一张有单位的资源账本", section "GQA改变共享接口").
+//
+// Layout of the work
+// ------------------
+// * Two CTAs per SM.  A CTA owns an equal share of the concatenated
+//   (b, h, 32-token block) list; a 32-token block is exactly one K group, so
+//   one K scale row serves the whole block.
+// * A CTA holds kNP warp pairs.  Each pair runs one 3-stage pipeline of bulk
+//   copies (cp.async.bulk, completion counted on an mbarrier) carrying, per
+//   block, 32 tokens of K codes (2 KB) and V codes (2 KB), the block's K
+//   scale row (512 B) and the tokens' V scales (512 B).
+//   - The S-warp (scores) folds the K scales into q once per block, unpacks
+//     K once for all four heads, sums lane partials through shared memory,
+//     runs the online softmax (m, z) and hands the V-warp each token's
+//     probabilities already multiplied by the token's V scales.  Scores are
+//     in log2 units (q carries scale * log2(e)), so exp is one ex2.
+//   - The V-warp (values) rescales its accumulators when m grows and adds
+//     p' * v for its 16 channels and four heads with packed f32x2 FMAs.
+//   Splitting the roles keeps each warp under 128 registers, so an SM runs
+//   16 warps.
+// * At the end of each (b, h) segment the pair states are merged in shared
+//   memory with the same rule and written as the output (segment covered
+//   whole by the CTA) or as a partial for the split merge kernel.
+//
+// Unpacking without a subtract
+// ----------------------------
+// A nibble n in mantissa bits [p, p+4) under exponent 0 reads as the float
+// 1 + n * 2^(p-23).  Shifting a code word left by 15, 7 or right by 1, 9 puts
+// the two nibbles of one byte at p = 15 and p = 19, so one LOP3 per code gives
+// f = 1 + n * eps with eps = 2^-8 for even channels and 2^-4 for odd ones,
+// and the two channels of a byte land in one f32x2 pair.  With q'' = q' / eps,
+// sum q'' f - sum q'' (1 + 7 eps) = sum q' (n - 7): the second sum is one
+// correction per block.  For V, u = (U - (1 + 7 eps) P) / eps with U = sum p' f
+// and P = sum p'.  Rounding error is amplified by at most 2^8 / 7.
+#include "kvq_internal.cuh"
+#include "plan.cuh"
+
+namespace kvq {
+namespace {
+
+typedef unsigned long long u64;       // one f32x2 value (low half = first float)
+
+constexpr int kD = 128;
+constexpr int kG = 4;                 // query heads per KV head
+constexpr int kTB = 32;               // tokens per block (one K group)
+constexpr int kNP = 4;                // warp pairs per CTA
+constexpr int kS = 3;                 // pipeline stages per pair
+constexpr int kThreads = 2 * kNP * 32;
+constexpr int kPartStride = 36;       // floats per token row of score partials (8 x 4 + pad)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kCorrEven = 1.f + 7.f / 256.f;
+constexpr float kCorrOdd = 1.f + 7.f / 16.f;
+
+struct Stage {
+  uint8_t kc[kTB * kD / 2];           // K codes, 64 B per token
+  uint8_t vc[kTB * kD / 2];           // V codes, 64 B per token
+  float ks[kD];                       // K scale row of the block's group
+  float vs[kTB][kD / 32];             // V scales, 4 per token
+};
+
+struct PairSmem {
+  Stage st[kS];
+  float part[2][kTB * kPartStride];   // score partials, double-buffered; part[0] holds the
+                                      // V-warp's U at merge time
+  float pv[kTB][20];                  // p' = p * s_v of token t, group g, head h at [t][4g + h];
+                                      // four entries pad the row
+  unsigned long long full[kS];        // copies landed
+  unsigned long long empty[kS];       // V-warp done with the stage
+  unsigned long long pfull[2];        // S-warp wrote part[i]
+  unsigned long long pempty[2];       // V-warp read part[i]
+};
+
+static_assert(sizeof(Stage) % 16 == 0, "stage alignment");
+static_assert(sizeof(PairSmem) % 16 == 0, "pair alignment");
+static_assert(kTB * kPartStride >= kG * kD, "U must fit in a partials buffer");
+
+struct DecodeParams {
+  const void* Q;
+  int q_dtype;
+  const uint8_t* k_codes;
+  const float* k_scales;
+  const uint8_t* v_codes;
+  const float* v_scales;
+  const int32_t* lengths;
+  int B, H, N_cap;
+  long long k_codes_head, k_scales_head, v_codes_head, v_scales_head;
+  float qscale;                       // scale * log2(e)
+  void* O;
+  float* partials;                    // [slots][kG][kD + 2]
+  int ctas;
+  unsigned int* err;
+};
+
+// shared memory after the pairs: qs [kG][kD] (swizzled), mm/mz [kNP][kG],
+// mP [kNP][4 groups][kG], pre [B + 1], len [B]
+size_t smem_bytes(int B) {
+  return sizeof(PairSmem) * kNP + sizeof(float) * (kG * kD + 2 * kNP * kG + kNP * 16) +
+         sizeof(int) * (2 * B + 1);
+}
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps in hardware (up to the hint, in ns) instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(unsigned long long* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(200000u)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: gives up after about two seconds, records KVQ_ERR_TIMEOUT and
+// returns false, so a lost completion ends the kernel instead of hanging it.
+__device__ __forceinline__ bool wait_bar(unsigned long long* bar, uint32_t parity,
+                                         unsigned int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 7u) == 0 && globaltimer() - t0 > 2000000000ull) {
+      record_error(err, KVQ_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// f32x2 values travel in 64-bit registers from the instruction that makes
+// them to the instruction that uses them, so no register-pair moves are
+// needed around the packed FMAs (u64 is declared with the constants).
+
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+  u64 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+  u64 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ u64 pack2(float lo, float hi) {
+  u64 d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+
+__device__ __forceinline__ float lo_f(u64 x) { return __uint_as_float(static_cast<uint32_t>(x)); }
+__device__ __forceinline__ float hi_f(u64 x) { return __uint_as_float(static_cast<uint32_t>(x >> 32)); }
+
+// The two channels of one code byte after a shift that puts them at bits
+// 15..18 and 19..22: (1 + n_even 2^-8, 1 + n_odd 2^-4) as one f32x2 value.
+__device__ __forceinline__ u64 nibble_pair(uint32_t a) {
+  u64 x;
+  asm("{.reg .b32 t0, t1;\n\t"
+      "lop3.b32 t0, %1, 0x00078000, 0x3F800000, 0xEA;\n\t"
+      "lop3.b32 t1, %1, 0x00780000, 0x3F800000, 0xEA;\n\t"
+      "mov.b64 %0, {t0, t1};}"
+      : "=l"(x)
+      : "r"(a));
+  return x;
+}
+
+// Channel pairs (16cs + 2i, 16cs + 2i + 1), i = 0..7, of one 64-bit code load.
+__device__ __forceinline__ void nibble_pairs(uint32_t w0, uint32_t w1, u64 f[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t w = i < 4 ? w0 : w1;
+    const int r = i & 3;
+    f[i] = nibble_pair(r == 0 ? (w << 15) : r == 1 ? (w << 7) : r == 2 ? (w >> 1) : (w >> 9));
+  }
+}
+
+// q of the segment lives in shared memory pre-scaled by 1/eps, with the four
+// 16-byte chunks of each lane's 16 channels rotated so the eight lanes of a
+// quarter warp hit eight different bank groups.
+__device__ __forceinline__ int qs_index(int h, int c) {
+  const int cs = c >> 4, j = (c >> 2) & 3;
+  return h * kD + cs * 16 + ((j ^ ((cs >> 1) & 3)) << 2) + (c & 3);
+}
+
+// ---------------------------------------------------------------------------
+// iteration over the CTA's block range
+// ---------------------------------------------------------------------------
+struct Seg {
+  int b, h, nb, jb, je;
+  long long gpos;                     // global index of block jb
+  bool valid;
+};
+
+__device__ __forceinline__ Seg first_seg(const int* pre, int B, int H, const CtaRange& cr) {
+  Seg s;
+  s.valid = cr.g0 < cr.g1;
+  if (!s.valid) return s;
+  s.b = find_seq(pre, B, H, cr.g0);
+  s.nb = pre[s.b + 1] - pre[s.b];
+  const long long off = cr.g0 - static_cast<long long>(H) * pre[s.b];
+  s.h = static_cast<int>(off / s.nb);
+  s.jb = static_cast<int>(off % s.nb);
+  s.je = static_cast<int>(min(static_cast<long long>(s.nb), s.jb + (cr.g1 - cr.g0)));
+  s.gpos = cr.g0;
+  return s;
+}
+
+__device__ __forceinline__ Seg next_seg(Seg s, const int* pre, int B, int H, const CtaRange& cr) {
+  s.gpos += s.je - s.jb;
+  if (s.gpos >= cr.g1) {
+    s.valid = false;
+    return s;
+  }
+  if (++s.h == H) {
+    s.h = 0;
+    ++s.b;
+    while (s.b < B && pre[s.b + 1] == pre[s.b]) ++s.b;
+  }
+  s.nb = pre[s.b + 1] - pre[s.b];
+  s.jb = 0;
+  s.je = static_cast<int>(min(static_cast<long long>(s.nb), cr.g1 - s.gpos));
+  return s;
+}
+
+struct Prod {
+  Seg seg;
+  int j;
+  bool valid;
+};
+
+__device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H, const CtaRange& cr,
+                                            int pair) {
+  while (p.valid && p.j >= p.seg.je) {
+    p.seg = next_seg(p.seg, pre, B, H, cr);
+    p.valid = p.seg.valid;
+    p.j = p.seg.jb + pair;
+  }
+  return p;
+}
+
+__device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem& ps, int stage, int b,
+                                            int h, int j, const int* slen) {
+  const long long head = static_cast<long long>(b) * p.H + h;
+  const int len = slen[b];
+  const int t0 = j * kTB;
+  const int nv = min(kTB, len - t0);
+  Stage& st = ps.st[stage];
+  unsigned long long* bar = &ps.full[stage];
+  mbar_expect_tx(bar, 144u * nv + 512u);
+  bulk_g2s(st.kc, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * (kD / 2),
+           nv * (kD / 2), bar);
+  bulk_g2s(st.vc, p.v_codes + head * p.v_codes_head + static_cast<long long>(t0) * (kD / 2),
+           nv * (kD / 2), bar);
+  bulk_g2s(st.ks, p.k_scales + head * p.k_scales_head + static_cast<long long>(j) * kD,
+           kD * sizeof(float), bar);
+  bulk_g2s(st.vs, p.v_scales + head * p.v_scales_head + static_cast<long long>(t0) * (kD / 32),
+           nv * 16, bar);
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  PairSmem* pairs = reinterpret_cast<PairSmem*>(smem_raw);
+  float* qs = reinterpret_cast<float*>(pairs + kNP);    // [kG][kD], swizzled, * 1/eps
+  float* mm = qs + kG * kD;                              // [kNP][kG] pair maxima
+  float* mz = mm + kNP * kG;                             // [kNP][kG] pair sums
+  float* mP = mz + kNP * kG;                             // [kNP][4][kG] pair sums of p'
+  int* pre = reinterpret_cast<int*>(mP + kNP * 16);      // [B + 1]
+  int* slen = pre + p.B + 1;                             // [B] lengths clamped to [0, N_cap]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool is_s = warp < kNP;                          // S-warp (scores) or V-warp (values)
+  const int pair = is_s ? warp : warp - kNP;
+  const int ts = lane >> 3, cs = lane & 7;
+  PairSmem& ps = pairs[pair];
+
+  if (warp == 0) warp_block_prefix(p.lengths, p.B, p.N_cap, kTB, pre);
+  for (int b = threadIdx.x; b < p.B; b += kThreads) slen[b] = clamp_len(p.lengths[b], p.N_cap);
+  if (is_s && lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kS; ++s) {
+      mbar_init(&ps.full[s], 1);
+      mbar_init(&ps.empty[s], 1);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ps.pfull[i], 1);
+      mbar_init(&ps.pempty[i], 1);
+    }
+  }
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncthreads();
+
+  const int H = p.H;
+  const CtaRange cr = cta_range(pre, p.B, H, p.ctas, blockIdx.x);
+  if (cr.g0 >= cr.g1) return;
+
+  Seg seg = first_seg(pre, p.B, H, cr);
+  Prod prod{seg, seg.jb + pair, true};
+  prod = prod_settle(prod, pre, p.B, H, cr, pair);
+  if (is_s) {
+    for (int s = 0; s < kS && prod.valid; ++s) {
+      if (lane == 0) issue_block(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
+      prod.j += kNP;
+      prod = prod_settle(prod, pre, p.B, H, cr, pair);
+    }
+  }
+
+  uint32_t k = 0;                                        // blocks this pair has consumed
+  while (seg.valid) {
+    const int b = seg.b, h = seg.h;
+    const long long head = static_cast<long long>(b) * H + h;
+    const long long qrow = static_cast<long long>(b) * H * kG + static_cast<long long>(h) * kG;
+    for (int i = threadIdx.x; i < kG * kD; i += kThreads) {
+      const float ie = (i & 1) ? 16.f : 256.f;           // 1/eps of the channel's parity
+      qs[qs_index(i / kD, i % kD)] = load_as_f32(p.Q, qrow * kD + i, p.q_dtype) * p.qscale * ie;
+    }
+    __syncthreads();
+    const int len = slen[b];
+
+    if (is_s) {
+      // ===================== S-warp: partial scores =====================
+      for (int j = seg.jb + pair; j < seg.je; j += kNP, ++k) {
+        const int stage = static_cast<int>(k % kS);
+        const int pb = static_cast<int>(k & 1u);
+        wait_bar(&ps.full[stage], (k / kS) & 1u, p.err);
+        const Stage& st = ps.st[stage];
+
+        // q'' = q * scale * log2e / eps * s_k, as channel pairs (16cs + 2i, +1)
+        u64 q2[kG][8];
+        u64 kcp[kG];
+        {
+          const ulonglong2* ksv = reinterpret_cast<const ulonglong2*>(st.ks + 16 * cs);
+          ulonglong2 kv2[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) kv2[jj] = ksv[jj];
+          const u64 corr = pack2(kCorrEven, kCorrOdd);
+#pragma unroll
+          for (int hh = 0; hh < kG; ++hh) {
+            u64 c2 = 0ull;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const ulonglong2 a2 = *reinterpret_cast<const ulonglong2*>(
+                  qs + hh * kD + cs * 16 + ((jj ^ ((cs >> 1) & 3)) << 2));
+              q2[hh][2 * jj] = mul2(a2.x, kv2[jj].x);
+              q2[hh][2 * jj + 1] = mul2(a2.y, kv2[jj].y);
+              c2 = fma2(q2[hh][2 * jj], corr, c2);
+              c2 = fma2(q2[hh][2 * jj + 1], corr, c2);
+            }
+            kcp[hh] = static_cast<u64>(__float_as_uint(-(lo_f(c2) + hi_f(c2))));
+          }
+        }
+        // the V-warp must have read this partial buffer's previous block
+        if (k >= 2) wait_bar(&ps.pempty[pb], ((k - 2) >> 1) & 1u, p.err);
+        float* part = ps.part[pb];
+#pragma unroll 2
+        for (int it = 0; it < kTB / 4; ++it) {
+          const int t = 4 * it + ts;
+          const uint2 kw = *reinterpret_cast<const uint2*>(st.kc + t * (kD / 2) + cs * 8);
+          u64 f[8];
+          nibble_pairs(kw.x, kw.y, f);
+          u64 acc[kG];
+#pragma unroll
+          for (int hh = 0; hh < kG; ++hh) {
+            acc[hh] = fma2(q2[hh][0], f[0], kcp[hh]);
+#pragma unroll
+            for (int i = 1; i < 8; ++i) acc[hh] = fma2(q2[hh][i], f[i], acc[hh]);
+          }
+          *reinterpret_cast<float4*>(part + t * kPartStride + cs * 4) =
+              make_float4(lo_f(acc[0]) + hi_f(acc[0]), lo_f(acc[1]) + hi_f(acc[1]),
+                          lo_f(acc[2]) + hi_f(acc[2]), lo_f(acc[3]) + hi_f(acc[3]));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ps.pfull[pb]);
+
+        // refill the stage of the previous block once the V-warp has released it
+        if (k > 0 && prod.valid) {
+          const uint32_t kp = k - 1;
+          const int sp = static_cast<int>(kp % kS);
+          wait_bar(&ps.empty[sp], (kp / kS) & 1u, p.err);
+          if (lane == 0) {
+            fence_proxy_async();
+            issue_block(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
+          }
+          prod.j += kNP;
+          prod = prod_settle(prod, pre, p.B, H, cr, pair);
+        }
+      }
+    } else {
+      // ===================== V-warp: softmax and values =====================
+      u64 u[kG][8];
+      float m[kG], z[kG], P[kG];                        // z: per token-lane; P: per (ts, cs) lane
+#pragma unroll
+      for (int hh = 0; hh < kG; ++hh) {
+        m[hh] = -INFINITY;
+        z[hh] = 0.f;
+        P[hh] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) u[hh][i] = 0ull;
+      }
+      const int g = cs >> 1;                            // V group of channels 16cs..16cs+15
+      for (int j = seg.jb + pair; j < seg.je; j += kNP, ++k) {
+        const int stage = static_cast<int>(k % kS);
+        const int pb = static_cast<int>(k & 1u);
+        wait_bar(&ps.full[stage], (k / kS) & 1u, p.err);
+        wait_bar(&ps.pfull[pb], (k >> 1) & 1u, p.err);
+        const Stage& st = ps.st[stage];
+        const int nvalid = min(kTB, len - j * kTB);
+
+        // scores of token `lane`: sum the eight channel-slice partials
+        float s[kG] = {0.f, 0.f, 0.f, 0.f};
+        const float* part = ps.part[pb];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 v = *reinterpret_cast<const float4*>(part + lane * kPartStride + 4 * i);
+          s[0] += v.x;
+          s[1] += v.y;
+          s[2] += v.z;
+          s[3] += v.w;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ps.pempty[pb]);
+
+        // online softmax over the block (log2 units)
+        const bool valid = lane < nvalid;
+        float a[kG], pr[kG];
+        bool grow = false;
+#pragma unroll
+        for (int hh = 0; hh < kG; ++hh) {
+          s[hh] = valid ? s[hh] : -INFINITY;
+          const float mn = fmaxf(m[hh], warp_max(s[hh]));
+          grow |= mn > m[hh];
+          a[hh] = ex2(m[hh] - mn);                      // 0 on the first block (m = -inf)
+          pr[hh] = valid ? ex2(s[hh] - mn) : 0.f;
+          z[hh] = fmaf(a[hh], z[hh], pr[hh]);
+          m[hh] = mn;
+        }
+        if (grow) {                                     // warp-uniform
+#pragma unroll
+          for (int hh = 0; hh < kG; ++hh) {
+            P[hh] *= a[hh];
+            const u64 a2 = pack2(a[hh], a[hh]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[hh][i] = mul2(u[hh][i], a2);
+          }
+        }
+        // p' = p * s_v of this lane's token for each V group, as (p', p') pairs
+        {
+          const float4 sv = *reinterpret_cast<const float4*>(st.vs[lane]);
+          const float svg[4] = {sv.x, sv.y, sv.z, sv.w};
+          const u64 p01 = pack2(pr[0], pr[1]), p23 = pack2(pr[2], pr[3]);
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const float sg = valid ? svg[gg] : 0.f;
+            const u64 s2 = pack2(sg, sg);
+            *reinterpret_cast<ulonglong2*>(&ps.pv[lane][4 * gg]) =
+                make_ulonglong2(mul2(p01, s2), mul2(p23, s2));
+          }
+        }
+        __syncwarp();
+
+        // values: lane (ts, cs), token 4*it + ts, channels 16cs..16cs+15
+#pragma unroll 2
+        for (int it = 0; it < kTB / 4; ++it) {
+          const int t = 4 * it + ts;
+          const float4 p4 = *reinterpret_cast<const float4*>(&ps.pv[t][4 * g]);
+          const uint2 vw = *reinterpret_cast<const uint2*>(st.vc + t * (kD / 2) + cs * 8);
+          u64 f[8];
+          nibble_pairs(vw.x, vw.y, f);
+          const u64 pp[kG] = {pack2(p4.x, p4.x), pack2(p4.y, p4.y), pack2(p4.z, p4.z),
+                              pack2(p4.w, p4.w)};
+          P[0] += p4.x;
+          P[1] += p4.y;
+          P[2] += p4.z;
+          P[3] += p4.w;
+#pragma unroll
+          for (int hh = 0; hh < kG; ++hh)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[hh][i] = fma2(pp[hh], f[i], u[hh][i]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ps.empty[stage]);
+      }
+
+      // pair state: z per token-lane; U and P per (ts, cs) lane -> reduce over ts
+#pragma unroll
+      for (int hh = 0; hh < kG; ++hh) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z[hh] += __shfl_xor_sync(0xffffffffu, z[hh], o);
+        P[hh] += __shfl_xor_sync(0xffffffffu, P[hh], 8);
+        P[hh] += __shfl_xor_sync(0xffffffffu, P[hh], 16);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int hh = 0; hh < kG; ++hh) {
+          mm[pair * kG + hh] = m[hh];
+          mz[pair * kG + hh] = z[hh];
+        }
+      }
+      if (ts == 0 && (cs & 1) == 0) {
+#pragma unroll
+        for (int hh = 0; hh < kG; ++hh) mP[(pair * 4 + g) * kG + hh] = P[hh];
+      }
+      float uf[kG][16];
+#pragma unroll
+      for (int hh = 0; hh < kG; ++hh)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float x = lo_f(u[hh][i]), y = hi_f(u[hh][i]);
+          x += __shfl_xor_sync(0xffffffffu, x, 8);
+          y += __shfl_xor_sync(0xffffffffu, y, 8);
+          x += __shfl_xor_sync(0xffffffffu, x, 16);
+          y += __shfl_xor_sync(0xffffffffu, y, 16);
+          uf[hh][2 * i] = x;
+          uf[hh][2 * i + 1] = y;
+        }
+      if (ts == 0) {
+#pragma unroll
+        for (int hh = 0; hh < kG; ++hh) {
+          float4* dst = reinterpret_cast<float4*>(ps.part[0] + hh * kD + 16 * cs);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_float4(uf[hh][4 * q], uf[hh][4 * q + 1], uf[hh][4 * q + 2], uf[hh][4 * q + 3]);
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- merge the pairs: thread -> (head, channel)
+    const bool whole = (seg.jb == 0) && (seg.je == seg.nb);
+    const long long slot = static_cast<long long>(blockIdx.x) + head;
+    for (int idx = threadIdx.x; idx < kG * kD; idx += kThreads) {
+      const int hh = idx / kD, c = idx % kD;
+      const float corr = (c & 1) ? kCorrOdd : kCorrEven;
+      const float ie = (c & 1) ? 16.f : 256.f;
+      float ms = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kNP; ++w)
+        if (mz[w * kG + hh] > 0.f) ms = fmaxf(ms, mm[w * kG + hh]);
+      float zt = 0.f, ut = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNP; ++w) {
+        const float zw = mz[w * kG + hh];
+        if (zw > 0.f) {
+          const float f = ex2(mm[w * kG + hh] - ms);
+          const float uw = (pairs[w].part[0][hh * kD + c] - corr * mP[(w * 4 + c / 32) * kG + hh]) * ie;
+          zt += f * zw;
+          ut += f * uw;
+        }
+      }
+      if (whole) {
+        store_from_f32(p.O, (qrow + hh) * kD + c, ut / zt, p.q_dtype);
+      } else {
+        float* part = p.partials + (slot * kG + hh) * (kD + 2);
+        if (c == 0) {
+          part[0] = ms * kLn2;
+          part[1] = zt;
+        }
+        part[2 + c] = ut;
+      }
+    }
+    __syncthreads();
+    seg = next_seg(seg, pre, p.B, H, cr);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+bool decode_applies(const AttendArgs& a) {
+  return a.g.bits == 4 && a.g.group == kTB && a.g.D == kD && a.Lq == 1 &&
+         a.H_q == kG * a.g.H_kv && smem_bytes(a.g.B) <= 113 * 1024;
+}
+
+int decode_ctas(const AttendArgs& a) {
+  const long long t_max = static_cast<long long>(a.g.B) * a.g.H_kv * ((a.g.N_cap + kTB - 1) / kTB);
+  long long ctas = a.splits > 0 ? a.splits : 2LL * (sm_count() > 0 ? sm_count() : 148);
+  if (ctas > t_max) ctas = t_max;
+  if (ctas < 1) ctas = 1;
+  return static_cast<int>(ctas);
+}
+
+size_t decode_workspace(const AttendArgs& a) {
+  return partial_slots(decode_ctas(a), a.g.B, a.g.H_kv) * kG * (kD + 2) * sizeof(float);
+}
+
+kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
+  const int ctas = decode_ctas(a);
+  const size_t smem = smem_bytes(a.g.B);
+  if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  DecodeParams p{};
+  p.Q = a.Q;
+  p.q_dtype = a.q_dtype;
+  p.k_codes = a.k_codes;
+  p.k_scales = a.k_scales;
+  p.v_codes = a.v_codes;
+  p.v_scales = a.v_scales;
+  p.lengths = a.lengths;
+  p.B = a.g.B;
+  p.H = a.g.H_kv;
+  p.N_cap = a.g.N_cap;
+  p.k_codes_head = static_cast<long long>(a.g.k_codes_head);
+  p.k_scales_head = static_cast<long long>(a.g.k_scales_head);
+  p.v_codes_head = static_cast<long long>(a.g.v_codes_head);
+  p.v_scales_head = static_cast<long long>(a.g.v_scales_head);
+  p.qscale = a.scale * kLog2e;
+  p.O = a.O;
+  p.partials = static_cast<float*>(a.workspace);
+  p.ctas = ctas;
+  p.err = error_word();
+  if (!p.err) return KVQ_ERR_CUDA;
+  decode_kernel<<<ctas, kThreads, smem, s>>>(p);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+
+  MergeArgs m{};
+  m.partials = p.partials;
+  m.lengths = a.lengths;
+  m.O = a.O;
+  m.o_dtype = a.q_dtype;
+  m.B = a.g.B;
+  m.H_kv = a.g.H_kv;
+  m.N_cap = a.g.N_cap;
+  m.BT = kTB;
+  m.ctas = ctas;
+  m.R = kG;
+  m.R_pad = kG;
+  m.D = kD;
+  m.G = kG;
+  m.Lq = 1;
+  return launch_merge(m, s);
+}
+
+const AttendImpl kDecode{"decode_gqa4_d128_b4g32", decode_applies, decode_workspace, decode_launch};
+
+}  // namespace
+
+const AttendImpl* decode_attend_impl() { return &kDecode; }
+
+}  // namespace kvq

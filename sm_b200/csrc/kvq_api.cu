@@ -130,10 +130,11 @@ kvq_status kvq_pack(const void* K, const void* V, kvq_dtype in_dtype, int32_t t0
                     const kvq_cache* cache, void* stream) {
   PackArgs a{};
   if (!make_geometry(cache, &a.g)) return KVQ_ERR_ARG;
-  if (!K || !V || !cache->k_codes || !cache->k_scales || !cache->v_codes || !cache->v_scales)
+  if ((!K && !V) || !cache->k_codes || !cache->k_scales || !cache->v_codes || !cache->v_scales)
     return KVQ_ERR_ARG;
   if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16) return KVQ_ERR_ARG;
-  if (t0 < 0 || t1 <= t0 || t1 > cache->N_cap || t0 % cache->group) return KVQ_ERR_ARG;
+  if (t0 < 0 || t1 <= t0 || t1 > cache->N_cap) return KVQ_ERR_ARG;
+  if (K && t0 % cache->group) return KVQ_ERR_ARG;
   const size_t esz = in_dtype == KVQ_F32 ? 4 : 2;
   if ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V)) % esz) return KVQ_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(cache->k_scales) | reinterpret_cast<uintptr_t>(cache->v_scales)) % 4)

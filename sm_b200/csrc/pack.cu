@@ -12,8 +12,16 @@
 namespace kvq {
 namespace {
 
-__device__ __forceinline__ unsigned quant_code(float x, float s, int qmax) {
-  float q = rintf(__fdiv_rn(x, s));
+// rint(x / s) with x / s correctly rounded first.  x * (1/s) is within a few
+// ulps of x / s, and |x / s| <= 127, so its error stays below 2^-15: unless it
+// lies within 2^-12 of a rounding tie it rounds to the same integer as the
+// correctly rounded quotient.  Near a tie (or if 1/s overflowed) the exact
+// IEEE division decides.
+__device__ __forceinline__ unsigned quant_code(float x, float s, float rs, int qmax) {
+  const float qa = x * rs;
+  float q = rintf(qa);
+  const float d = fabsf(qa - q);
+  if (!(d < 0.5f - 0.000244140625f)) q = rintf(__fdiv_rn(x, s));
   q = fminf(fmaxf(q, -static_cast<float>(qmax)), static_cast<float>(qmax));
   return static_cast<unsigned>(static_cast<int>(q) + qmax);
 }
@@ -36,7 +44,7 @@ struct PackParams {
 // each channel; the group's codes are g*D consecutive entries of the
 // flattened Np x D code matrix, so a 4-bit group owns whole bytes (g even).
 __global__ void __launch_bounds__(256) pack_k_kernel(PackParams p) {
-  extern __shared__ float s_x[];                   // [g][D] then scale[D]
+  extern __shared__ float s_x[];                   // [g][D], then scale[D], 1/scale[D]
   const int gi = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = p.group, D = p.D;
   const int qmax = p.bits == 4 ? 7 : 127;
@@ -56,6 +64,7 @@ __global__ void __launch_bounds__(256) pack_k_kernel(PackParams p) {
     for (int tt = 0; tt < g; ++tt) amax = fmaxf(amax, fabsf(s_x[tt * D + d]));
     const float sc = group_scale(amax, qmax);
     s_scale[d] = sc;
+    s_scale[D + d] = __frcp_rn(sc);
     p.scales[head * p.scales_head + kgroup * D + d] = sc;
   }
   __syncthreads();
@@ -64,13 +73,14 @@ __global__ void __launch_bounds__(256) pack_k_kernel(PackParams p) {
   if (p.bits == 4) {
     for (int jb = threadIdx.x; jb < g * D / 2; jb += blockDim.x) {
       const int f = 2 * jb;
-      const unsigned lo = quant_code(s_x[f], s_scale[f % D], qmax);
-      const unsigned hi = quant_code(s_x[f + 1], s_scale[(f + 1) % D], qmax);
+      const int d0 = f % D, d1 = (f + 1) % D;
+      const unsigned lo = quant_code(s_x[f], s_scale[d0], s_scale[D + d0], qmax);
+      const unsigned hi = quant_code(s_x[f + 1], s_scale[d1], s_scale[D + d1], qmax);
       out[code0 / 2 + jb] = static_cast<uint8_t>(lo | (hi << 4));
     }
   } else {
     for (int f = threadIdx.x; f < g * D; f += blockDim.x)
-      out[code0 + f] = static_cast<uint8_t>(quant_code(s_x[f], s_scale[f % D], qmax));
+      out[code0 + f] = static_cast<uint8_t>(quant_code(s_x[f], s_scale[f % D], s_scale[D + f % D], qmax));
   }
 }
 
@@ -95,6 +105,7 @@ __global__ void __launch_bounds__(256) pack_v_kernel(PackParams p) {
     if (d < D) amax = fmaxf(amax, fabsf(load_as_f32(p.X, in_base + d, p.dtype)));
   }
   const float sc = group_scale(amax, qmax);
+  const float rs = __frcp_rn(sc);
   const long long tok = static_cast<long long>(p.t0) + tt;
   p.scales[head * p.scales_head + tok * ng + gj] = sc;
   const long long code0 = tok * p.Dp + d0;
@@ -103,13 +114,55 @@ __global__ void __launch_bounds__(256) pack_v_kernel(PackParams p) {
     for (int e = 0; e < g; e += 2) {
       const float x0 = d0 + e < D ? load_as_f32(p.X, in_base + d0 + e, p.dtype) : 0.f;
       const float x1 = d0 + e + 1 < D ? load_as_f32(p.X, in_base + d0 + e + 1, p.dtype) : 0.f;
-      out[(code0 + e) / 2] = static_cast<uint8_t>(quant_code(x0, sc, qmax) | (quant_code(x1, sc, qmax) << 4));
+      out[(code0 + e) / 2] =
+          static_cast<uint8_t>(quant_code(x0, sc, rs, qmax) | (quant_code(x1, sc, rs, qmax) << 4));
     }
   } else {
     for (int e = 0; e < g; ++e) {
       const float x = d0 + e < D ? load_as_f32(p.X, in_base + d0 + e, p.dtype) : 0.f;
-      out[code0 + e] = static_cast<uint8_t>(quant_code(x, sc, qmax));
+      out[code0 + e] = static_cast<uint8_t>(quant_code(x, sc, rs, qmax));
     }
+  }
+}
+
+// V, D = 128 and groups of 32: one warp per token row.  Lane l holds features
+// 4l..4l+3 (one 16-byte load), the 8 lanes of a group reduce the group max
+// with shuffles, and the lane writes its 4 codes (2 bytes, or 4 at 8 bits).
+__global__ void __launch_bounds__(256) pack_v128_kernel(PackParams p) {
+  const long long rows = static_cast<long long>(p.B) * p.H * p.T;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const int qmax = p.bits == 4 ? 7 : 127;
+  float x[4];
+  if (p.dtype == KVQ_F32) {
+    const float4 v = reinterpret_cast<const float4*>(p.X)[row * 32 + lane];
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  } else {
+    const uint2 v = reinterpret_cast<const uint2*>(p.X)[row * 32 + lane];
+    x[0] = __uint_as_float(v.x << 16);
+    x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(v.y << 16);
+    x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  }
+  float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+  const float sc = group_scale(amax, qmax);
+  const float rs = __frcp_rn(sc);
+  const long long head = row / p.T;
+  const long long tok = static_cast<long long>(p.t0) + row % p.T;
+  if ((lane & 7) == 0) p.scales[head * p.scales_head + tok * 4 + (lane >> 3)] = sc;
+  unsigned c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = quant_code(x[i], sc, rs, qmax);
+  uint8_t* out = p.codes + head * p.codes_head;
+  if (p.bits == 4) {
+    reinterpret_cast<uint16_t*>(out + tok * 64)[lane] =
+        static_cast<uint16_t>(c[0] | (c[1] << 4) | (c[2] << 8) | (c[3] << 12));
+  } else {
+    reinterpret_cast<uint32_t*>(out + tok * 128)[lane] = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
   }
 }
 
@@ -118,31 +171,45 @@ __global__ void __launch_bounds__(256) pack_v_kernel(PackParams p) {
 kvq_status launch_pack(const PackArgs& a, cudaStream_t s) {
   const Geometry& g = a.g;
   const int T = a.t1 - a.t0;
-  const size_t smem = (static_cast<size_t>(g.group) * g.D + g.D) * sizeof(float);
-  if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
   if (g.B > 65535 || g.H_kv > 65535) return KVQ_ERR_UNSUPPORTED;
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(pack_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return KVQ_ERR_CUDA;
+  if (a.K) {
+    const size_t smem = (static_cast<size_t>(g.group) * g.D + 2 * g.D) * sizeof(float);
+    if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
+    if (smem > 48 * 1024) {
+      if (cudaFuncSetAttribute(pack_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    }
+    PackParams pk{a.K, a.in_dtype, a.t0, T, g.bits, g.group, g.B, g.H_kv, g.D, g.Dp,
+                  static_cast<long long>(g.k_codes_head), static_cast<long long>(g.k_scales_head),
+                  a.k_codes, a.k_scales};
+    const dim3 kgrid((T + g.group - 1) / g.group, g.H_kv, g.B);
+    pack_k_kernel<<<kgrid, 256, smem, s>>>(pk);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   }
-  PackParams pk{a.K, a.in_dtype, a.t0, T, g.bits, g.group, g.B, g.H_kv, g.D, g.Dp,
-                static_cast<long long>(g.k_codes_head), static_cast<long long>(g.k_scales_head),
-                a.k_codes, a.k_scales};
-  const dim3 kgrid((T + g.group - 1) / g.group, g.H_kv, g.B);
-  pack_k_kernel<<<kgrid, 256, smem, s>>>(pk);
-  count_launch();
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
-
-  PackParams pv{a.V, a.in_dtype, a.t0, T, g.bits, g.group, g.B, g.H_kv, g.D, g.Dp,
-                static_cast<long long>(g.v_codes_head), static_cast<long long>(g.v_scales_head),
-                a.v_codes, a.v_scales};
-  const long long vthreads = static_cast<long long>(g.B) * g.H_kv * T * (g.Dp / g.group);
-  const long long vblocks = (vthreads + 255) / 256;
-  if (vblocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
-  pack_v_kernel<<<static_cast<unsigned>(vblocks), 256, 0, s>>>(pv);
-  count_launch();
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  if (a.V) {
+    PackParams pv{a.V, a.in_dtype, a.t0, T, g.bits, g.group, g.B, g.H_kv, g.D, g.Dp,
+                  static_cast<long long>(g.v_codes_head), static_cast<long long>(g.v_scales_head),
+                  a.v_codes, a.v_scales};
+    const size_t esz = a.in_dtype == KVQ_F32 ? 4 : 2;
+    const bool fast = g.D == 128 && g.group == 32 &&
+                      (reinterpret_cast<uintptr_t>(a.V) % (4 * esz)) == 0 &&
+                      (reinterpret_cast<uintptr_t>(a.v_codes) % 4) == 0;
+    if (fast) {
+      const long long rows = static_cast<long long>(g.B) * g.H_kv * T;
+      const long long blocks = (rows + 7) / 8;
+      if (blocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
+      pack_v128_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(pv);
+    } else {
+      const long long vthreads = static_cast<long long>(g.B) * g.H_kv * T * (g.Dp / g.group);
+      const long long vblocks = (vthreads + 255) / 256;
+      if (vblocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
+      pack_v_kernel<<<static_cast<unsigned>(vblocks), 256, 0, s>>>(pv);
+    }
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  }
   return KVQ_OK;
 }
 

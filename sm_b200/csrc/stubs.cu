@@ -2,6 +2,6 @@
 #include "kvq_internal.cuh"
 
 namespace kvq {
-const AttendImpl* decode_attend_impl() { return nullptr; }
+
 const AttendImpl* chunk_attend_impl() { return nullptr; }
 }  // namespace kvq

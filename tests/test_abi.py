@@ -83,7 +83,7 @@ def test_pack_range_rules():
     assert call(0, 65) == 1          # beyond capacity
     assert call(-32, 8) == 1
     assert call(0, 8, dt=7) == 1     # unknown dtype
-    assert call(0, 8, kp=0) == 1     # NULL input
+    assert K.lib.kvq_pack(None, None, K.KVQ_F32, 0, 8, ctypes.byref(c), None) == 1  # both NULL
     assert call(0, 8, kp=0x1002) == 3  # misaligned float32 input
 
 

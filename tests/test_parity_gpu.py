@@ -60,6 +60,39 @@ def test_pack_all_zero_and_ties(sm):
     assert_head_packed_equal(cache, 0, 0, O.pack_k(ties, 4, 8), O.pack_v(ties, 4, 8))
 
 
+def test_pack_ties_d128(sm):
+    """Width 128, group 32 (the warp-per-row V kernel): every group holds +-7
+    (scale exactly 1) and half-integers, so the quotient lands on rounding
+    ties and must round half to even; also a few random rows."""
+    rng = np.random.default_rng(12)
+    x = rng.integers(-14, 15, size=(1, 2, 64, 128)).astype(np.float32) / 2
+    x[..., ::32] = 7.0
+    x[..., 1, :] = rng.standard_normal(128).astype(np.float32)
+    cache = pack_gpu(sm, x, x, 4, 32)
+    for h in range(2):
+        assert_head_packed_equal(cache, 0, h, O.pack_k(x[0, h], 4, 32), O.pack_v(x[0, h], 4, 32))
+    cache8 = pack_gpu(sm, x * 127 / 7, x * 127 / 7, 8, 32)
+    for h in range(2):
+        y = (x[0, h] * 127 / 7).astype(np.float32)
+        assert_head_packed_equal(cache8, 0, h, O.pack_k(y, 8, 32), O.pack_v(y, 8, 32))
+
+
+def test_pack_halves_separately(sm):
+    """K alone over a group-aligned range, then V alone over one token (the
+    decode-step append), equals packing both together."""
+    rng = np.random.default_rng(13)
+    k = rng.standard_normal((2, 3, 64, 128)).astype(np.float32)
+    v = rng.standard_normal((2, 3, 64, 128)).astype(np.float32)
+    both = pack_gpu(sm, k, v, 4, 32)
+    sep = sm.PackedCache(2, 3, 64, 128, 4, 32, DEV)
+    sm.pack(to_dev(k), None, sep)
+    for t in range(64):
+        sm.pack(None, to_dev(v[:, :, t:t + 1]), sep, t0=t)
+    for a, b in ((both.k_codes, sep.k_codes), (both.v_codes, sep.v_codes),
+                 (both.k_scales, sep.k_scales), (both.v_scales, sep.v_scales)):
+        assert torch.equal(a, b)
+
+
 def test_pack_append_matches_whole(sm):
     """Packing [0, 64) then [64, 100) then re-packing the tail group from its
     start, [96, 130), gives the bytes of a whole [0, 130) pack."""
