@@ -84,21 +84,30 @@ def append_bytes(B, H_kv, D, k_tokens, v_tokens=1, bits=4, group=32, in_bytes=4)
 # environment
 # ---------------------------------------------------------------------------
 
-def measured_peaks():
+def measured_peaks(kind: str = "hbm"):
+    """(peak, source): HBM GB/s or dense bf16 TFLOP/s (burst) from the
+    measured file, else the fallback figures."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs" if kind == "hbm" else "bf16_tflops"]), "measured"
     except Exception:
-        return 6650.0, "fallback"
+        return (6650.0 if kind == "hbm" else 1590.0), "fallback"
 
 
-def recorded_traffic(kernel_src: str):
+PROFILE_FOR = {
+    "decode_gqa": "attend_decode_gqa_b32_ctx4096.md",
+    "long_context": "attend_decode_long_context_b8.md",
+    "chunk": "attend_chunk_b4_lq64_ctx16384.md",
+}
+
+
+def recorded_traffic(kernel_src: str, workload: str = "decode_gqa"):
     """Per-launch DRAM bytes of the attend kernel from the committed ncu
     summary, or None when the kernel source changed since the capture."""
     import hashlib
-    summary = os.path.join(ROOT, "profiles", "attend_decode_gqa_b32_ctx4096.md")
+    summary = os.path.join(ROOT, "profiles", PROFILE_FOR.get(workload, ""))
     try:
         text = open(summary, encoding="utf-8").read()
         src = open(kernel_src, "rb").read()
@@ -185,24 +194,27 @@ def blas_threads() -> int:
 
 
 def oracle_step_sample(heads, q, k, v, lengths, meta, prepacked):
-    """One oracle decode step on the sampled (b, h_kv) heads: pack the tail
-    group, decode the head, attend its query heads.  Returns bytes counted
-    with the same accounting as the GPU step."""
+    """One oracle step on the sampled (b, h_kv) heads: pack the group(s) of
+    the step's new tokens, decode the head, attend its query heads' rows.
+    Returns bytes counted with the same accounting as the GPU step."""
     import oracle as O
     grp = meta["H_q"] // meta["H_kv"]
-    bits, g, d = meta["bits"], meta["group"], meta["D"]
+    bits, g, d, lq = meta["bits"], meta["group"], meta["D"], meta["Lq"]
+    uniform = bool(np.all(np.asarray(lengths) == meta["N"]))
     nbytes = 0
     for (b, h) in heads:
         n = int(lengths[b])
-        t0 = (n - 1) // g * g
-        pk_tail = O.pack_k(k[b, h, t0:n], bits, g)
-        pv_new = O.pack_v(v[b, h, n - 1:n], bits, g)
+        t0 = (n - lq) // g * g
+        if uniform:
+            O.pack_k(k[b, h, t0:n], bits, g)
+            O.pack_v(v[b, h, n - lq:n], bits, g)
         pk, pv = prepacked[(b, h)]
         kh, vh = O.unpack_matrix(pk), O.unpack_matrix(pv)
-        _ = (pk_tail, pv_new)
-        O.attend_gqa_heads(q[b, h * grp:(h + 1) * grp, 0], kh, vh, n, 1.0)
-        nbytes += (attend_bytes(1, grp, 1, d, [n], bits, g)
-                   + append_bytes(1, 1, d, n - t0, 1, bits, g))
+        rows = q[b, h * grp:(h + 1) * grp].reshape(grp * lq, d)
+        O.attend_gqa_heads(rows, kh, vh, n, 1.0)
+        nbytes += attend_bytes(1, grp, 1, d, [n], bits, g, lq=lq)
+        if uniform:
+            nbytes += append_bytes(1, 1, d, n - t0, lq, bits, g)
     return nbytes
 
 
@@ -234,11 +246,19 @@ def run_kvq(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    q_np, k_np, v_np, lens_np, meta = W.gqa_case(WORKLOAD, SEED + rank)
+    workload = args.workload
+    q_np, k_np, v_np, lens_np, meta = W.gqa_case(workload, SEED + rank)
     q_np = torch.from_numpy(q_np).to(torch.bfloat16).float().numpy()
-    B, H_q, H_kv, D, N = meta["B"], meta["H_q"], meta["H_kv"], meta["D"], meta["N"]
-    bits, g = meta["bits"], meta["group"]
-    t0 = (N - 1) // g * g                       # tail group start (the new token is N-1)
+    B, H_q, H_kv, D, N, Lq = meta["B"], meta["H_q"], meta["H_kv"], meta["D"], meta["N"], meta["Lq"]
+    bits = args.bits if args.bits else (meta["bits"] if isinstance(meta["bits"], int) else 4)
+    meta["bits"] = bits
+    g = meta["group"]
+    uniform = bool(np.all(lens_np == N))
+    # the step's append: the K group(s) holding the new tokens (re-packed from a
+    # float32 recent-token window) and the new tokens' V rows; only when every
+    # sequence has the same length, since one kvq_pack call covers one range
+    t0 = (N - Lq) // g * g
+    v0 = N - Lq
 
     caches = []
     kd = torch.from_numpy(k_np).to(dev)
@@ -247,21 +267,22 @@ def run_kvq(args, rank, world, local_rank):
         c = K.PackedCache(B, H_kv, N, D, bits, g, dev)
         K.pack(kd, vd, c)
         caches.append(c)
-    win_k = kd[:, :, t0:N].contiguous()          # K of the tail group (recent-token window)
-    new_v = vd[:, :, N - 1:N].contiguous()       # V of the new token
+    win_k = kd[:, :, t0:N].contiguous()          # K of the new tokens' groups (recent-token window)
+    new_v = vd[:, :, v0:N].contiguous()          # V of the new tokens
     del kd, vd
     qd = torch.from_numpy(q_np).to(dev).to(torch.bfloat16)
     lens = torch.from_numpy(lens_np).to(dev)
     out = torch.empty_like(qd)
-    ws_need = K.workspace_size(caches[0], H_q, 1)
+    ws_need = K.workspace_size(caches[0], H_q, Lq)
     ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
     K.check(dev)
 
     def step(i):
         c = caches[i & 1]
-        K.pack(win_k, None, c, t0=t0)
-        K.pack(None, new_v, c, t0=N - 1)
+        if uniform:
+            K.pack(win_k, None, c, t0=t0)
+            K.pack(None, new_v, c, t0=v0)
         K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
 
     def attend_only(i):
@@ -325,7 +346,7 @@ def run_kvq(args, rank, world, local_rank):
     # end-to-end through the public API (direct calls, no graphs) with the
     # step's inputs copied from pinned host buffers and the output read back
     q_host = torch.from_numpy(q_np).to(torch.bfloat16).pin_memory()
-    kv_host_k = win_k[:, :, -1:].cpu().pin_memory()
+    kv_host_k = win_k[:, :, -Lq:].cpu().pin_memory()
     kv_host_v = new_v.cpu().pin_memory()
     o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -338,20 +359,22 @@ def run_kvq(args, rank, world, local_rank):
     for i in range(args.steps):
         c = caches[i & 1]
         qd.copy_(q_host, non_blocking=True)
-        win_k[:, :, -1:].copy_(kv_host_k, non_blocking=True)
-        new_v.copy_(kv_host_v, non_blocking=True)
-        K.pack(win_k, None, c, t0=t0)
-        K.pack(None, new_v, c, t0=N - 1)
+        if uniform:
+            win_k[:, :, -Lq:].copy_(kv_host_k, non_blocking=True)
+            new_v.copy_(kv_host_v, non_blocking=True)
+            K.pack(win_k, None, c, t0=t0)
+            K.pack(None, new_v, c, t0=v0)
         K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
         o_host.copy_(out, non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
-    h2d = q_host.numel() * 2 + (kv_host_k.numel() + kv_host_v.numel()) * 4
+    h2d = q_host.numel() * 2 + ((kv_host_k.numel() + kv_host_v.numel()) * 4 if uniform else 0)
     d2h = o_host.numel() * 2
 
-    step_bytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g) + append_bytes(B, H_kv, D, N - t0, 1, bits, g)
-    abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g)
+    abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g, lq=Lq)
+    step_bytes = abytes + (append_bytes(B, H_kv, D, N - t0, Lq, bits, g) if uniform else 0)
+    attend_flops = 4 * H_q * Lq * D * int(np.sum(lens_np.astype(np.int64)))
     t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -363,33 +386,44 @@ def run_kvq(args, rank, world, local_rank):
         value = world * step_bytes / (per_step_ms * 1e-3) / 1e9
         e2e_value = world * step_bytes / (e2e_max / args.steps * 1e-3) / 1e9
         att_ms = statistics.mean(attend_ms)
-        achieved = abytes / (att_ms * 1e-3) / 1e9
-        peak, peak_kind = measured_peaks()
-        kname = K.kernel_name(caches[0], H_q, 1)
+        tensor = workload == "chunk"
+        if tensor:
+            achieved = attend_flops / (att_ms * 1e-3) / 1e12
+            peak, peak_kind = measured_peaks("tensor")
+        else:
+            achieved = abytes / (att_ms * 1e-3) / 1e9
+            peak, peak_kind = measured_peaks("hbm")
+        kname = K.kernel_name(caches[0], H_q, Lq)
         src = os.path.join(ROOT, "sm_b200", "csrc",
-                           "attend_decode.cu" if kname.startswith("decode") else "attend_generic.cu")
+                           "attend_decode.cu" if kname.startswith("decode") else
+                           "attend_chunk.cu" if kname.startswith("chunk") else "attend_generic.cu")
         res = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 6),
             "us_per_step": round(per_step_ms * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "storage": "u4 codes + f32 scales (group 32), bf16 Q/O",
+            "dtype": "f32", "storage": f"u{bits} codes + f32 scales (group {g}), bf16 Q/O",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": B, "H_q": H_q, "H_kv": H_kv, "d_h": D,
-                       "context": N, "bits": bits, "group": g, "lq": 1,
-                       "step": "append (re-pack the K group of the new token, pack its V row) + attend",
-                       "l2": "inputs larger than L2: 2 packed caches of 168 MB used in turn",
+            "config": {"workload": workload, "B": B, "H_q": H_q, "H_kv": H_kv, "d_h": D,
+                       "context": N if uniform else "per-sequence", "lengths_sum": int(np.sum(lens_np)),
+                       "bits": bits, "group": g, "lq": Lq,
+                       "step": ("append (re-pack the K group(s) of the new tokens, pack their V rows) + attend"
+                                if uniform else "attend (per-sequence lengths; no shared append range)"),
+                       "l2": f"inputs larger than L2: 2 packed caches of {caches[0].nbytes() / 1e6:.0f} MB used in turn",
                        "parallelism": f"independent batch per GPU x{world}",
                        "attend_kernel": kname, "step_bytes": step_bytes,
-                       "launch": "CUDA graph per step (append + attend)"},
+                       "launch": "CUDA graph per step"},
             "pct_of_8tbs": round(100 * value / world / 8000.0, 2),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "peak_source": f"hbm_gbs of {peak_kind}",
+            "roofline": {"bound": "tensor" if tensor else "hbm", "achieved": round(achieved, 1 if not tensor else 2),
+                         "peak": peak, "unit": "TFLOP/s" if tensor else "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "peak_source": ("bf16_tflops (burst) of " if tensor else "hbm_gbs of ") + peak_kind,
                          "kernel": f"kvq_attend ({kname})", "attend_us": round(att_ms * 1e3, 3),
                          "timing": "attend-only CUDA-graph replays, same caches in turn",
                          "algorithmic_bytes_per_launch": abytes,
-                         "traffic": recorded_traffic(src)},
+                         "algorithmic_flops_per_launch": attend_flops,
+                         "attend_gbs": round(abytes / (att_ms * 1e-3) / 1e9, 1),
+                         "traffic": recorded_traffic(src, workload)},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_max / args.steps * 1e3, 3)},
             "gpu_launches": int(launches),
@@ -408,6 +442,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=64,
                     help="(b, h_kv) heads in the oracle's timed sample")
+    ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD,
+                    help="the decode GQA workload is the headline; the others are for study")
+    ap.add_argument("--bits", type=int, choices=[4, 8], default=0,
+                    help="code width for the chunk workload (default 4)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -419,9 +457,11 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        q, k, v, lens, meta = W.gqa_case(WORKLOAD, SEED)
+        q, k, v, lens, meta = W.gqa_case(args.workload, SEED)
         import torch
         q = torch.from_numpy(q).to(torch.bfloat16).float().numpy()
+        if not isinstance(meta["bits"], int):
+            meta["bits"] = args.bits or 4
         per_step = max(4, args.cpu_heads // 4)
         total, times = 0, []
         for _ in range(args.warmup):
@@ -437,9 +477,11 @@ def main():
             "ms_per_step": round(1e3 * sum(times) / len(times), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": meta["B"], "H_q": meta["H_q"],
-                       "H_kv": meta["H_kv"], "d_h": meta["D"], "context": meta["N"],
-                       "bits": meta["bits"], "group": meta["group"], "lq": 1},
+            "config": {"workload": args.workload, "B": meta["B"], "H_q": meta["H_q"],
+                       "H_kv": meta["H_kv"], "d_h": meta["D"],
+                       "context": meta["N"] if bool(np.all(lens == meta["N"])) else "per-sequence",
+                       "lengths_sum": int(np.sum(lens)),
+                       "bits": meta["bits"], "group": meta["group"], "lq": meta["Lq"]},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(),
                              "kind": "oracle",

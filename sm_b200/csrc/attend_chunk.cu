@@ -1,0 +1,916 @@
+// Multi-query chunk attention on the tcgen05 tensor cores: D = 128, 4- or 8-bit
+// codes in groups of 32, bf16 Q/O, 128 or 256 query rows per KV head (the
+// GQA group's heads times the chunk's queries), non-causal over the whole
+// valid cache ("注意力分塊：不保存完整分數矩陣，如何保持結果？", opening section: the
+// queries read the whole existing context).
+//
+// Per 128-token block the packed K/V bytes are decoded -- (code - qmax) *
+// scale, as "KV分组打包：4-bit到底省了多少？" section "一个字节里到底装了什么"
+// defines it -- into bf16 tiles in shared memory, S = Q K^T runs on the
+// tensor cores into tensor memory (TMEM), the online softmax turns S into P
+// in place, and O += P V runs on the tensor cores again with P read straight
+// from TMEM.  The running (m, z, u) rule of "Block KV decoding: less workspace,
+// more time" (section "Do not average independently normalized blocks") is
+// applied per query row; u lives in TMEM.
+//
+// Rescaling is lazy: a row's reference maximum only moves (and O, z are
+// multiplied by exp(m_old - m_new)) when a block's maximum exceeds it by more
+// than 8 in log2 units.  Any reference that never falls more than that below
+// the true running maximum gives the same u / z in exact arithmetic, and the
+// exponentials stay <= 2^8, well inside bf16/fp32 range.
+//
+// Warp roles (16 warps):
+//   0        producer: cp.async.bulk of the packed codes + scales, one unit
+//            per K or V half of a block, into a ring of 54 KB (5 units at
+//            4 bits, 3 at 8 bits).  Unit order K(0), K(1), V(0), K(2), V(1),
+//            ...: the K decode runs one block ahead of the V decode.
+//   1        MMA issuer (one thread) and TMEM owner (512 columns)
+//   2        Q loader: a 2-D TMA copy with 128-byte swizzle of the segment's
+//            Q rows, once the previous segment's Q K^T products are done
+//   4..7     softmax of query rows 0..127 (TMEM lanes 0..127, warp w owns
+//            lanes 32*(w%4)..+31); 8..11 the same for rows 128..255
+//   12..15   decode: warp w converts the 32-token group w-12 of each K unit
+//            (into one of two K tiles) and the same tokens of each V unit
+//   3        idle
+// The MMA order per block k is QK0(k) QK1(k) | PV0(k) QK0(k+1) PV1(k)
+// QK1(k+1) | ...: while one row tile is in the softmax the tensor cores work
+// on the other.  A Q K^T product overwrites the S columns that hold the
+// previous block's P, so it waits for that tile's P V product to complete.
+//
+// TMEM columns: S/P of row tile t at [128 t, 128 t + 128), O of row tile t at
+// [256 + 128 t, 256 + 128 t + 128).  P (bf16) overwrites the first 64 columns
+// of its S tile.
+//
+// Shared memory tiles use the 128-byte-swizzled UMMA layout: a row of 64 bf16
+// (128 B) with its 16-byte chunks XOR-permuted by (row % 8), eight-row atoms
+// of 1 KB -- the layout a TMA copy with 128-byte swizzle writes.  Q tiles and
+// the K tiles are K-major (rows = query rows / tokens, contiguous = features);
+// the V tile is stored the same way (rows = tokens) and read as an MN-major
+// operand.  Each 128-feature row is split in two 64-feature halves of 16 KB.
+#include <cuda.h>
+
+#include "kvq_internal.cuh"
+#include "plan.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kBT = 128;              // tokens per block
+constexpr int kThreads = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLazy = 8.f;          // log2 units a row max may outrun its reference
+
+// shared-memory carve (bytes from a 1024-aligned base)
+constexpr int kTileHalf = kBT * 128;              // 16 KB: 128 rows x 64 bf16
+constexpr int kOffQ = 0;                          // 2 row tiles x 2 halves
+constexpr int kOffK = 4 * kTileHalf;              // 2 K tiles (double buffer)
+constexpr int kOffV = kOffK + 4 * kTileHalf;      // 1 V tile
+constexpr int kOffRing = kOffV + 2 * kTileHalf;   // 160 KB
+constexpr int kRingBytes = 54 * 1024;
+constexpr int kMaxUnits = 5;
+constexpr int kOffBar = kOffRing + kRingBytes;
+constexpr int kNumBars = 24;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // TMEM base slot
+constexpr int kOffPre = kOffMisc + 16;            // int pre[B + 1], len[B]
+
+enum Bar {
+  RING_FULL = 0,                 // [kMaxUnits]
+  RING_EMPTY = 5,                // [kMaxUnits]
+  K_READY = 10,                  // [2]
+  K_FREE = 12,                   // [2]
+  V_READY = 14,
+  V_FREE = 15,
+  Q_READY = 16,
+  Q_FREE = 17,
+  S_FULL = 18,                   // [2]
+  P_FULL = 20,                   // [2]
+  PV_DONE = 22,                  // [2]
+};
+constexpr int kDecodeWarps = 4;
+
+struct ChunkParams {
+  const uint8_t* k_codes;
+  const float* k_scales;
+  const uint8_t* v_codes;
+  const float* v_scales;
+  const int32_t* lengths;
+  int bits, B, H, N_cap, G, Lq, R, NT;   // R = G * Lq rows per (b, h), NT = R / 128 row tiles
+  long long k_codes_head, k_scales_head, v_codes_head, v_scales_head;
+  float qscale;                          // scale * log2(e)
+  __nv_bfloat16* O;
+  float* partials;                       // [slots][kD + 2][R]: m, z, u (feature-major)
+  int ctas;
+  unsigned int* err;
+};
+
+size_t smem_bytes(int B) { return 1024 + kOffPre + sizeof(int) * (2 * B + 1); }
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t su(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(100000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: after about two seconds record KVQ_ERR_TIMEOUT, raise the
+// CTA's abort flag and go on; once the flag is up every later wait of the CTA
+// returns at once, so the kernel always reaches its end (and frees its tensor
+// memory) within a few seconds.
+__device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, unsigned int* err, volatile int* abort_flag) {
+  if (mbar_try(bar, parity)) return;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(bar, parity)) {
+    if (*abort_flag) return;
+    if (globaltimer() - t0 > 2000000000ull) {
+      record_error(err, KVQ_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return;
+    }
+  }
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+#define KVQ_LD32(r, taddr)                                                                             \
+  asm volatile(                                                                                        \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"  \
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                        \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),        \
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),      \
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),      \
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                           \
+      : "r"(taddr))
+
+#define KVQ_ST32(taddr, r)                                                                             \
+  asm volatile(                                                                                        \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"    \
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),          \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), \
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),    \
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),   \
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]))
+
+#define KVQ_ST16(taddr, r)                                                                              \
+  asm volatile(                                                                                         \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"     \
+      "%15,%16};" ::"r"(taddr),                                                                         \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),  \
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]))
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// UMMA shared-memory descriptor: 128-byte swizzle, 1 KB eight-row atoms.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor, kind::f16: bf16 A and B, f32 accumulate, M = 128.
+__host__ __device__ constexpr uint32_t instr_desc(int n, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a swizzled 64-wide half.
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// 8 nibble codes of one word (feature e in bits 4e..4e+3) to the exact floats
+// code - 7.  Each nibble is masked into mantissa bits 12..15 or 16..19 of 1.0,
+// which makes 1 + n/2048 or 1 + n/128, and one FMA takes that to n - 7.
+__device__ __forceinline__ void nibbles_to_f32(uint32_t w, float (&v)[8]) {
+  const uint32_t a = w << 12, b = w << 4, c = w >> 8, d = w >> 12;
+  auto lo = [](uint32_t x) { return __uint_as_float(0x3F800000u | (x & 0x0000F000u)); };
+  auto hi = [](uint32_t x) { return __uint_as_float(0x3F800000u | (x & 0x000F0000u)); };
+  v[0] = fmaf(lo(a), 2048.f, -2055.f);
+  v[1] = fmaf(hi(a), 128.f, -135.f);
+  v[2] = fmaf(lo(b), 2048.f, -2055.f);
+  v[3] = fmaf(hi(b), 128.f, -135.f);
+  v[4] = fmaf(hi(w), 128.f, -135.f);
+  v[5] = fmaf(lo(c), 2048.f, -2055.f);
+  v[6] = fmaf(hi(c), 128.f, -135.f);
+  v[7] = fmaf(hi(d), 128.f, -135.f);
+}
+
+// 4 byte codes of one word to the exact floats code - 127: the byte goes into
+// the low mantissa bits of 2^23 with one byte permute.
+__device__ __forceinline__ void bytes_to_f32(uint32_t w, float (&v)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + k)) - 8388735.f;
+}
+
+// ---------------------------------------------------------------------------
+// the CTA's blocks, one at a time (same walk as the plan)
+// ---------------------------------------------------------------------------
+struct Seg {
+  int b, h, nb, jb, je;
+  long long gpos;
+  bool valid;
+};
+__device__ __forceinline__ Seg first_seg(const int* pre, int B, int H, const CtaRange& cr) {
+  Seg s;
+  s.valid = cr.g0 < cr.g1;
+  if (!s.valid) return s;
+  s.b = find_seq(pre, B, H, cr.g0);
+  s.nb = pre[s.b + 1] - pre[s.b];
+  const long long off = cr.g0 - static_cast<long long>(H) * pre[s.b];
+  s.h = static_cast<int>(off / s.nb);
+  s.jb = static_cast<int>(off % s.nb);
+  s.je = static_cast<int>(min(static_cast<long long>(s.nb), s.jb + (cr.g1 - cr.g0)));
+  s.gpos = cr.g0;
+  return s;
+}
+__device__ __forceinline__ Seg next_seg(Seg s, const int* pre, int B, int H, const CtaRange& cr) {
+  s.gpos += s.je - s.jb;
+  if (s.gpos >= cr.g1) {
+    s.valid = false;
+    return s;
+  }
+  if (++s.h == H) {
+    s.h = 0;
+    ++s.b;
+    while (s.b < B && pre[s.b + 1] == pre[s.b]) ++s.b;
+  }
+  s.nb = pre[s.b + 1] - pre[s.b];
+  s.jb = 0;
+  s.je = static_cast<int>(min(static_cast<long long>(s.nb), cr.g1 - s.gpos));
+  return s;
+}
+
+// A position in the CTA's block list: segment (one (b, h)) and block j in it.
+struct Cursor {
+  Seg seg;
+  int j;
+  bool valid;
+  __device__ __forceinline__ void start(const int* pre, int B, int H, const CtaRange& cr) {
+    seg = first_seg(pre, B, H, cr);
+    j = seg.jb;
+    valid = seg.valid && seg.jb < seg.je;
+  }
+  __device__ __forceinline__ void next(const int* pre, int B, int H, const CtaRange& cr) {
+    if (++j == seg.je) {
+      seg = next_seg(seg, pre, B, H, cr);
+      j = seg.jb;
+      valid = seg.valid;
+    }
+  }
+  __device__ __forceinline__ bool first() const { return j == seg.jb; }
+  __device__ __forceinline__ bool last() const { return j + 1 == seg.je; }
+};
+
+// Row maximum of one S tile row (128 columns in TMEM), scaled by qscale:
+// max over the valid columns of s * qscale, taken as max(sgn * s) * |qscale|.
+template <bool kNeg>
+__device__ __forceinline__ float row_max(uint32_t s_col, int nv, float aq) {
+  float mb = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < 4; c += 2) {
+    uint32_t sa[32], sb[32];
+    KVQ_LD32(sa, s_col + 32u * c);
+    KVQ_LD32(sb, s_col + 32u * (c + 1));
+    tmem_wait_ld();
+    if (nv >= kBT) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float x = kNeg ? -__uint_as_float(sa[e]) : __uint_as_float(sa[e]);
+        const float y = kNeg ? -__uint_as_float(sb[e]) : __uint_as_float(sb[e]);
+        mb = fmaxf(mb, fmaxf(x, y));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float x = kNeg ? -__uint_as_float(sa[e]) : __uint_as_float(sa[e]);
+        const float y = kNeg ? -__uint_as_float(sb[e]) : __uint_as_float(sb[e]);
+        if (32 * c + e < nv) mb = fmaxf(mb, x);
+        if (32 * (c + 1) + e < nv) mb = fmaxf(mb, y);
+      }
+    }
+  }
+  return mb * aq;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ CUtensorMap qmap, ChunkParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw_addr = su(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  unsigned char* sm = smem_raw + (base - raw_addr);
+  int* pre = reinterpret_cast<int*>(sm + kOffPre);
+  int* slen = pre + p.B + 1;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+  const uint32_t bar0 = base + kOffBar;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = p.H;
+  const int cb = kD * p.bits / 8;                         // code bytes per token
+  const int unit_bytes = kBT * cb + 2048;                 // codes + scales of a K or V half-block
+  const uint32_t nu = static_cast<uint32_t>(min(kMaxUnits, kRingBytes / unit_bytes));
+
+  if (warp == 0) warp_block_prefix(p.lengths, p.B, p.N_cap, kBT, pre);
+  for (int b = threadIdx.x; b < p.B; b += kThreads) slen[b] = clamp_len(p.lengths[b], p.N_cap);
+  if (threadIdx.x == 32) {
+    *abort_flag = 0;
+    for (uint32_t u = 0; u < nu; ++u) {
+      mbar_init(bar(RING_FULL + u), 1);
+      mbar_init(bar(RING_EMPTY + u), kDecodeWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(K_READY + i), kDecodeWarps);
+      mbar_init(bar(K_FREE + i), 1);
+      mbar_init(bar(S_FULL + i), 1);
+      mbar_init(bar(P_FULL + i), 4);
+      mbar_init(bar(PV_DONE + i), 1);
+    }
+    mbar_init(bar(V_READY), kDecodeWarps);
+    mbar_init(bar(V_FREE), 1);
+    mbar_init(bar(Q_READY), 1);
+    mbar_init(bar(Q_FREE), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(base + kOffMisc),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + kOffMisc);
+
+  // sequences with a length outside 1..N_cap: report; rows of sequences with
+  // no valid key are zero (no block of theirs exists)
+  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+    const int raw = p.lengths[b];
+    if (threadIdx.x == 0 && (raw < 1 || raw > p.N_cap)) record_error(p.err, KVQ_ERR_LENGTH);
+    if (slen[b] == 0) {
+      const long long row0 = static_cast<long long>(b) * H * p.R;
+      for (long long i = threadIdx.x; i < static_cast<long long>(H) * p.R * kD; i += kThreads)
+        p.O[row0 * kD + i] = __float2bfloat16_rn(0.f);
+    }
+  }
+
+  const CtaRange cr = cta_range(pre, p.B, H, p.ctas, blockIdx.x);
+  if (cr.g0 < cr.g1) {
+    if (warp == 0) {
+      // ======================= producer =======================
+      if (lane == 0) {
+        Cursor kc, vc;
+        kc.start(pre, p.B, H, cr);
+        vc.start(pre, p.B, H, cr);
+        uint32_t n = 0;
+        auto unit = [&](const Cursor& c, bool is_v) {
+          const uint32_t slot = n % nu;
+          if (n >= nu) wait_bar(bar(RING_EMPTY + slot), ((n / nu) - 1) & 1u, p.err, abort_flag);
+          const long long head = static_cast<long long>(c.seg.b) * H + c.seg.h;
+          const int t0 = c.j * kBT;
+          const int nv = min(kBT, slen[c.seg.b] - t0);
+          const uint32_t dst = base + kOffRing + slot * unit_bytes;
+          const uint32_t fb = bar(RING_FULL + slot);
+          if (!is_v) {
+            const int ng = (nv + 31) / 32;
+            mbar_expect_tx(fb, static_cast<uint32_t>(nv * cb + ng * kD * 4));
+            bulk_g2s(dst, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * cb, nv * cb, fb);
+            bulk_g2s(dst + kBT * cb, p.k_scales + head * p.k_scales_head + static_cast<long long>(t0 / 32) * kD,
+                     ng * kD * 4, fb);
+          } else {
+            mbar_expect_tx(fb, static_cast<uint32_t>(nv * cb + nv * 16));
+            bulk_g2s(dst, p.v_codes + head * p.v_codes_head + static_cast<long long>(t0) * cb, nv * cb, fb);
+            bulk_g2s(dst + kBT * cb, p.v_scales + head * p.v_scales_head + static_cast<long long>(t0) * 4, nv * 16,
+                     fb);
+          }
+          ++n;
+        };
+        if (kc.valid) {
+          unit(kc, false);
+          kc.next(pre, p.B, H, cr);
+        }
+        while (vc.valid) {
+          if (kc.valid) {
+            unit(kc, false);
+            kc.next(pre, p.B, H, cr);
+          }
+          unit(vc, true);
+          vc.next(pre, p.B, H, cr);
+        }
+      }
+    } else if (warp == 1) {
+      // ======================= MMA issuer =======================
+      if (lane == 0) {
+        const uint32_t idesc_qk = instr_desc(kBT, false);
+        const uint32_t idesc_pv = instr_desc(kD, true);
+        auto qk = [&](int t, uint32_t k) {
+          const uint32_t kt = base + kOffK + (k & 1u) * 2 * kTileHalf;
+          for (int i = 0; i < kD / 16; ++i) {
+            const uint32_t q_addr = base + kOffQ + t * 2 * kTileHalf + (i >> 2) * kTileHalf + (i & 3) * 32;
+            const uint32_t k_addr = kt + (i >> 2) * kTileHalf + (i & 3) * 32;
+            mma_ss(tmem + 128u * t, smem_desc(q_addr, 16, 1024), smem_desc(k_addr, 16, 1024), idesc_qk, i > 0);
+          }
+          mma_commit(bar(S_FULL + t));
+        };
+        auto pv = [&](int t, uint32_t k, bool first) {
+          wait_bar(bar(P_FULL + t), k & 1u, p.err, abort_flag);
+          tc_fence_after();
+          for (int i = 0; i < kBT / 16; ++i) {
+            const uint32_t v_addr = base + kOffV + i * 16 * 128;
+            mma_ts(tmem + 256u + 128u * t, tmem + 128u * t + 8u * i, smem_desc(v_addr, kTileHalf, 1024), idesc_pv,
+                   (!first) || (i > 0));
+          }
+          mma_commit(bar(PV_DONE + t));
+        };
+        Cursor c;
+        c.start(pre, p.B, H, cr);
+        uint32_t sq = 0;
+        // block 0: Q of the first segment, its K tile, both Q K^T products
+        wait_bar(bar(Q_READY), sq & 1u, p.err, abort_flag);
+        ++sq;
+        wait_bar(bar(K_READY), 0u, p.err, abort_flag);
+        tc_fence_after();
+        for (int t = 0; t < p.NT; ++t) qk(t, 0);
+        mma_commit(bar(K_FREE));
+        if (c.last()) mma_commit(bar(Q_FREE));
+        Cursor cn = c;
+        cn.next(pre, p.B, H, cr);
+        for (uint32_t k = 0; c.valid; ++k) {
+          const bool boundary = cn.valid && cn.first();
+          wait_bar(bar(V_READY), k & 1u, p.err, abort_flag);
+          tc_fence_after();
+          pv(0, k, c.first());
+          if (cn.valid && !boundary) {
+            wait_bar(bar(K_READY + ((k + 1) & 1u)), ((k + 1) >> 1) & 1u, p.err, abort_flag);
+            wait_bar(bar(PV_DONE), k & 1u, p.err, abort_flag);
+            tc_fence_after();
+            qk(0, k + 1);
+          }
+          if (p.NT == 2) pv(1, k, c.first());
+          mma_commit(bar(V_FREE));
+          if (cn.valid) {
+            if (boundary) {
+              wait_bar(bar(Q_READY), sq & 1u, p.err, abort_flag);
+              ++sq;
+              wait_bar(bar(K_READY + ((k + 1) & 1u)), ((k + 1) >> 1) & 1u, p.err, abort_flag);
+              wait_bar(bar(PV_DONE), k & 1u, p.err, abort_flag);
+              tc_fence_after();
+              qk(0, k + 1);
+            }
+            if (p.NT == 2) {
+              wait_bar(bar(PV_DONE + 1), k & 1u, p.err, abort_flag);
+              tc_fence_after();
+              qk(1, k + 1);
+            }
+            mma_commit(bar(K_FREE + ((k + 1) & 1u)));
+            if (cn.last()) mma_commit(bar(Q_FREE));
+          }
+          c = cn;
+          cn.next(pre, p.B, H, cr);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 2) {
+      // ======================= Q loader =======================
+      if (lane == 0) {
+        uint32_t s = 0;
+        for (Seg seg = first_seg(pre, p.B, H, cr); seg.valid; seg = next_seg(seg, pre, p.B, H, cr), ++s) {
+          if (s > 0) wait_bar(bar(Q_FREE), (s - 1) & 1u, p.err, abort_flag);
+          const int row0 = (seg.b * H * p.G + seg.h * p.G) * p.Lq;
+          mbar_expect_tx(bar(Q_READY), static_cast<uint32_t>(p.NT * 2 * kTileHalf));
+          for (int t = 0; t < p.NT; ++t)
+            for (int half = 0; half < 2; ++half)
+              tma_load_2d(base + kOffQ + (2 * t + half) * kTileHalf, &qmap, 64 * half, row0 + 128 * t, bar(Q_READY));
+        }
+      }
+    } else if (warp >= 12) {
+      // ======================= decode K/V to bf16 tiles =======================
+      const int wk = warp - 12;                          // 32-token group of each unit
+      const uint32_t qmask = static_cast<uint32_t>(cb / 16 - 1);   // 16-byte chunks per token - 1
+      const int tsh = p.bits == 4 ? 2 : 3;               // lane = token * chunks + chunk
+      const int q = lane & qmask;
+      const int tt = lane >> tsh;
+      Cursor kc, vc;
+      kc.start(pre, p.B, H, cr);
+      vc.start(pre, p.B, H, cr);
+      uint32_t n = 0, kb = 0, vb = 0;
+      auto decode = [&](const Cursor& c, bool is_v) {
+        const uint32_t slot = n % nu;
+        wait_bar(bar(RING_FULL + slot), (n / nu) & 1u, p.err, abort_flag);
+        if (!is_v && kb >= 2) wait_bar(bar(K_FREE + (kb & 1u)), ((kb >> 1) - 1) & 1u, p.err, abort_flag);
+        if (is_v && vb >= 1) wait_bar(bar(V_FREE), (vb - 1) & 1u, p.err, abort_flag);
+        const unsigned char* u = sm + kOffRing + slot * unit_bytes;
+        unsigned char* dst = sm + (is_v ? kOffV : kOffK + (kb & 1u) * 2 * kTileHalf);
+        const int nv = min(kBT, slen[c.seg.b] - c.j * kBT);
+        const bool gvalid = wk * 32 < nv;
+        if (p.bits == 4) {
+          float ks[32];
+          if (!is_v && gvalid) {
+            const float4* s4 = reinterpret_cast<const float4*>(u + kBT * cb) + (wk * kD + 32 * q) / 4;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 v4 = s4[i];
+              ks[4 * i] = v4.x, ks[4 * i + 1] = v4.y, ks[4 * i + 2] = v4.z, ks[4 * i + 3] = v4.w;
+            }
+          }
+#pragma unroll 1
+          for (int it = 0; it < 4; ++it) {
+            const int t = 32 * wk + 8 * it + tt;
+            uint4 o[4] = {};
+            if (t < nv) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * cb + 16 * q);
+              const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+              const float vs = is_v ? reinterpret_cast<const float*>(u + kBT * cb)[4 * t + q] : 0.f;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                float f[8];
+                nibbles_to_f32(w[i], f);
+                uint32_t h[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float s0 = is_v ? vs : ks[8 * i + 2 * e];
+                  const float s1 = is_v ? vs : ks[8 * i + 2 * e + 1];
+                  h[e] = pack_bf16(f[2 * e] * s0, f[2 * e + 1] * s1);
+                }
+                o[i] = make_uint4(h[0], h[1], h[2], h[3]);
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int ch = 4 * q + i;
+              *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
+            }
+          }
+        } else {
+          float ks[16];
+          if (!is_v && gvalid) {
+            const float4* s4 = reinterpret_cast<const float4*>(u + kBT * cb) + (wk * kD + 16 * q) / 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 v4 = s4[i];
+              ks[4 * i] = v4.x, ks[4 * i + 1] = v4.y, ks[4 * i + 2] = v4.z, ks[4 * i + 3] = v4.w;
+            }
+          }
+#pragma unroll 1
+          for (int it = 0; it < 8; ++it) {
+            const int t = 32 * wk + 4 * it + tt;
+            uint4 o[2] = {};
+            if (t < nv) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * cb + 16 * q);
+              const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+              const float vs = is_v ? reinterpret_cast<const float*>(u + kBT * cb)[4 * t + (q >> 1)] : 0.f;
+              uint32_t h[8];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                float f[4];
+                bytes_to_f32(w[i], f);
+                const float s0 = is_v ? vs : ks[4 * i], s1 = is_v ? vs : ks[4 * i + 1];
+                const float s2 = is_v ? vs : ks[4 * i + 2], s3 = is_v ? vs : ks[4 * i + 3];
+                h[2 * i] = pack_bf16(f[0] * s0, f[1] * s1);
+                h[2 * i + 1] = pack_bf16(f[2] * s2, f[3] * s3);
+              }
+              o[0] = make_uint4(h[0], h[1], h[2], h[3]);
+              o[1] = make_uint4(h[4], h[5], h[6], h[7]);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int ch = 2 * q + i;
+              *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
+            }
+          }
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(is_v ? V_READY : K_READY + (kb & 1u)));
+          mbar_arrive(bar(RING_EMPTY + slot));
+        }
+        ++n;
+        if (is_v) ++vb; else ++kb;
+      };
+      if (kc.valid) {
+        decode(kc, false);
+        kc.next(pre, p.B, H, cr);
+      }
+      while (vc.valid) {
+        if (kc.valid) {
+          decode(kc, false);
+          kc.next(pre, p.B, H, cr);
+        }
+        decode(vc, true);
+        vc.next(pre, p.B, H, cr);
+      }
+    } else if (warp >= 4) {
+      // ======================= softmax: one query row per thread =======================
+      const int tile = (warp - 4) >> 2;
+      const int r = ((warp & 3) << 5) + lane;            // TMEM lane = row within the tile
+      const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const uint32_t s_col = tmem + lane_addr + 128u * tile;
+      const uint32_t o_col = tmem + lane_addr + 256u + 128u * tile;
+      const bool neg = p.qscale < 0.f;
+      const float aq = fabsf(p.qscale);
+      if (tile < p.NT) {
+        float m_ref = -INFINITY, z = 0.f;
+        Cursor c;
+        c.start(pre, p.B, H, cr);
+        for (uint32_t k = 0; c.valid; ++k, c.next(pre, p.B, H, cr)) {
+          if (c.first()) {
+            m_ref = -INFINITY;
+            z = 0.f;
+          }
+          wait_bar(bar(S_FULL + tile), k & 1u, p.err, abort_flag);
+          tc_fence_after();
+          const int nv = min(kBT, slen[c.seg.b] - c.j * kBT);
+          const float mb = neg ? row_max<true>(s_col, nv, aq) : row_max<false>(s_col, nv, aq);
+          // lazy rescale: move the reference only when the block max outruns it
+          const bool need = mb > m_ref + kLazy;
+          const float m_new = need ? mb : m_ref;
+          const float a = need ? ex2(m_ref - m_new) : 1.f;  // 0 on the first block
+          z *= a;
+          m_ref = m_new;
+          if (__any_sync(0xffffffffu, need) && !c.first()) {
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t orr[32];
+              KVQ_LD32(orr, o_col + 32u * cc);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * a);
+              KVQ_ST32(o_col + 32u * cc, orr);
+            }
+          }
+          // p = exp2(s * qscale - m_ref) as bf16, written over the S columns
+          const float nm = -m_ref;
+#pragma unroll 1
+          for (int cc = 0; cc < 4; cc += 2) {
+            uint32_t sa[32], sb[32];
+            KVQ_LD32(sa, s_col + 32u * cc);
+            KVQ_LD32(sb, s_col + 32u * (cc + 1));
+            tmem_wait_ld();
+            uint32_t pa[16], pb[16];
+            if (nv >= kBT) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float p0 = ex2(fmaf(__uint_as_float(sa[2 * e]), p.qscale, nm));
+                const float p1 = ex2(fmaf(__uint_as_float(sa[2 * e + 1]), p.qscale, nm));
+                const float p2 = ex2(fmaf(__uint_as_float(sb[2 * e]), p.qscale, nm));
+                const float p3 = ex2(fmaf(__uint_as_float(sb[2 * e + 1]), p.qscale, nm));
+                z += (p0 + p1) + (p2 + p3);
+                pa[e] = pack_bf16(p0, p1);
+                pb[e] = pack_bf16(p2, p3);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int t0 = 32 * cc + 2 * e, t1 = t0 + 32;
+                const float p0 = t0 < nv ? ex2(fmaf(__uint_as_float(sa[2 * e]), p.qscale, nm)) : 0.f;
+                const float p1 = t0 + 1 < nv ? ex2(fmaf(__uint_as_float(sa[2 * e + 1]), p.qscale, nm)) : 0.f;
+                const float p2 = t1 < nv ? ex2(fmaf(__uint_as_float(sb[2 * e]), p.qscale, nm)) : 0.f;
+                const float p3 = t1 + 1 < nv ? ex2(fmaf(__uint_as_float(sb[2 * e + 1]), p.qscale, nm)) : 0.f;
+                z += (p0 + p1) + (p2 + p3);
+                pa[e] = pack_bf16(p0, p1);
+                pb[e] = pack_bf16(p2, p3);
+              }
+            }
+            KVQ_ST16(s_col + 16u * cc, pa);
+            KVQ_ST16(s_col + 16u * (cc + 1), pb);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(P_FULL + tile));
+          if (c.last()) {
+            // the segment's last P V product must be done before O is read
+            wait_bar(bar(PV_DONE + tile), k & 1u, p.err, abort_flag);
+            tc_fence_after();
+            const bool whole = (c.seg.jb == 0) && (c.seg.je == c.seg.nb);
+            const long long head = static_cast<long long>(c.seg.b) * H + c.seg.h;
+            const long long row = (static_cast<long long>(c.seg.b) * H * p.G + static_cast<long long>(c.seg.h) * p.G) *
+                                      p.Lq + tile * 128 + r;
+            float* part = p.partials + (static_cast<long long>(blockIdx.x) + head) * (kD + 2) * p.R + tile * 128 + r;
+            if (!whole) {
+              part[0] = m_ref * kLn2;
+              part[p.R] = z;
+            }
+            const float inv = 1.f / z;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t orr[32];
+              KVQ_LD32(orr, o_col + 32u * cc);
+              tmem_wait_ld();
+              if (whole) {
+                uint32_t ob[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                  ob[e] = pack_bf16(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
+                uint4* dst = reinterpret_cast<uint4*>(p.O + row * kD + 32 * cc);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq)
+                  dst[qq] = make_uint4(ob[4 * qq], ob[4 * qq + 1], ob[4 * qq + 2], ob[4 * qq + 3]);
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) part[static_cast<long long>(2 + 32 * cc + e) * p.R] = __uint_as_float(orr[e]);
+              }
+            }
+            tc_fence_before();
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+int rows_per_head(const AttendArgs& a) { return (a.H_q / a.g.H_kv) * a.Lq; }
+
+bool chunk_applies(const AttendArgs& a) {
+  const int R = rows_per_head(a);
+  return a.g.D == kD && a.g.group == 32 && (a.g.bits == 4 || a.g.bits == 8) && a.q_dtype == KVQ_BF16 &&
+         (R == 128 || R == 256) && (reinterpret_cast<uintptr_t>(a.Q) & 15u) == 0 &&
+         static_cast<long long>(a.g.B) * a.H_q * a.Lq < (1LL << 31) && smem_bytes(a.g.B) <= 227 * 1024;
+}
+
+int chunk_ctas(const AttendArgs& a) {
+  const long long t_max = static_cast<long long>(a.g.B) * a.g.H_kv * ((a.g.N_cap + kBT - 1) / kBT);
+  long long ctas = a.splits > 0 ? a.splits : (sm_count() > 0 ? sm_count() : 148);
+  if (ctas > t_max) ctas = t_max;
+  if (ctas < 1) ctas = 1;
+  return static_cast<int>(ctas);
+}
+
+size_t chunk_workspace(const AttendArgs& a) {
+  return partial_slots(chunk_ctas(a), a.g.B, a.g.H_kv) * rows_per_head(a) * (kD + 2) * sizeof(float);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_tiled() {
+  static EncodeTiled fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiled>(nullptr);
+    return reinterpret_cast<EncodeTiled>(f);
+  }();
+  return fn;
+}
+
+// Q as a 2-D bf16 tensor [B * H_q * Lq rows][128], boxes of 128 rows x 64
+// features written with the 128-byte swizzle the UMMA descriptors expect.
+bool make_q_map(const AttendArgs& a, CUtensorMap* map) {
+  const EncodeTiled enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD),
+                              static_cast<cuuint64_t>(a.g.B) * a.H_q * a.Lq};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.Q), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
+  const int ctas = chunk_ctas(a);
+  const size_t smem = smem_bytes(a.g.B);
+  if (cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  CUtensorMap qmap;
+  if (!make_q_map(a, &qmap)) return KVQ_ERR_CUDA;
+  ChunkParams p{};
+  p.k_codes = a.k_codes;
+  p.k_scales = a.k_scales;
+  p.v_codes = a.v_codes;
+  p.v_scales = a.v_scales;
+  p.lengths = a.lengths;
+  p.bits = a.g.bits;
+  p.B = a.g.B;
+  p.H = a.g.H_kv;
+  p.N_cap = a.g.N_cap;
+  p.G = a.H_q / a.g.H_kv;
+  p.Lq = a.Lq;
+  p.R = rows_per_head(a);
+  p.NT = p.R / 128;
+  p.k_codes_head = static_cast<long long>(a.g.k_codes_head);
+  p.k_scales_head = static_cast<long long>(a.g.k_scales_head);
+  p.v_codes_head = static_cast<long long>(a.g.v_codes_head);
+  p.v_scales_head = static_cast<long long>(a.g.v_scales_head);
+  p.qscale = a.scale * kLog2e;
+  p.O = static_cast<__nv_bfloat16*>(a.O);
+  p.partials = static_cast<float*>(a.workspace);
+  p.ctas = ctas;
+  p.err = error_word();
+  if (!p.err) return KVQ_ERR_CUDA;
+  chunk_kernel<<<ctas, kThreads, smem, s>>>(qmap, p);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+
+  MergeArgs m{};
+  m.partials = p.partials;
+  m.lengths = a.lengths;
+  m.O = a.O;
+  m.o_dtype = a.q_dtype;
+  m.B = a.g.B;
+  m.H_kv = a.g.H_kv;
+  m.N_cap = a.g.N_cap;
+  m.BT = kBT;
+  m.ctas = ctas;
+  m.R = p.R;
+  m.R_pad = p.R;
+  m.D = kD;
+  m.G = p.G;
+  m.Lq = a.Lq;
+  m.feature_major = true;
+  return launch_merge(m, s);
+}
+
+const AttendImpl kChunk{"chunk_tcgen05_d128", chunk_applies, chunk_workspace, chunk_launch};
+
+}  // namespace
+
+const AttendImpl* chunk_attend_impl() { return &kChunk; }
+
+}  // namespace kvq

@@ -74,13 +74,15 @@ __device__ __forceinline__ int seq_blocks(int len, int n_cap, int bt) {
 
 // Merge partial states of a split (b, h) and write the output rows.
 struct MergeArgs {
-  const float* partials;           // [slots][R_pad][D + 2] : m, z, u[D]
+  const float* partials;           // row-major: [slots][R_pad][D + 2] : m, z, u[D]
+                                   // feature-major: [slots][D + 2][R_pad]
   const int32_t* lengths;
   void* O;
   int o_dtype;
   int B, H_kv, N_cap, BT, ctas;
   int R, R_pad, D;                 // rows per (b,h) and the padded row count of a slot
   int G, Lq;                       // query heads per KV head, rows per query head
+  bool feature_major;              // partial layout (rows contiguous per field)
 };
 kvq_status launch_merge(const MergeArgs& a, cudaStream_t s);
 

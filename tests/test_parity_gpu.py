@@ -198,6 +198,19 @@ def test_gqa_multi_query_rows(sm):
     _check_gqa(sm, q, k, v, lens, 4, 32, 1.0)
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("lq", [32, 64])
+def test_chunk_tensor_core_ragged(sm, bits, lq):
+    """The tcgen05 chunk kernel (128 or 256 query rows per KV head): ragged
+    lengths that end inside a 128-token block and inside a K group, a
+    sequence shorter than one block, and several splits."""
+    q, k, v, lens = _gqa_case(3, 8, 2, 700, 128, [700, 300, 77], lq=lq, seed=21 + bits, bits=bits)
+    cache = pack_gpu(sm, k, v, bits, 32)
+    assert sm.kernel_name(cache, 8, lq).startswith("chunk")
+    for splits in (0, 1, 5):
+        _check_gqa(sm, q, k, v, lens, bits, 32, 1.0, splits=splits)
+
+
 def test_repeat_is_bit_identical(sm):
     q, k, v, lens = _gqa_case(2, 8, 2, 300, 128, [300, 200], seed=6)
     cache = pack_gpu(sm, k, v, 4, 32)
