@@ -49,6 +49,7 @@
 // operand.  Each 128-feature row is split in two 64-feature halves of 16 KB.
 #include <cuda.h>
 
+#include "f32x2.cuh"
 #include "kvq_internal.cuh"
 #include "plan.cuh"
 
@@ -195,6 +196,19 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                           \
       : "r"(taddr))
 
+// the same, into r[o .. o + 31] of a larger register array
+#define KVQ_LD32_AT(r, o, taddr)                                                                       \
+  asm volatile(                                                                                        \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"  \
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                        \
+      : "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]),   \
+        "=r"(r[o + 6]), "=r"(r[o + 7]), "=r"(r[o + 8]), "=r"(r[o + 9]), "=r"(r[o + 10]), "=r"(r[o + 11]), \
+        "=r"(r[o + 12]), "=r"(r[o + 13]), "=r"(r[o + 14]), "=r"(r[o + 15]), "=r"(r[o + 16]),             \
+        "=r"(r[o + 17]), "=r"(r[o + 18]), "=r"(r[o + 19]), "=r"(r[o + 20]), "=r"(r[o + 21]),             \
+        "=r"(r[o + 22]), "=r"(r[o + 23]), "=r"(r[o + 24]), "=r"(r[o + 25]), "=r"(r[o + 26]),             \
+        "=r"(r[o + 27]), "=r"(r[o + 28]), "=r"(r[o + 29]), "=r"(r[o + 30]), "=r"(r[o + 31])              \
+      : "r"(taddr))
+
 #define KVQ_ST32(taddr, r)                                                                             \
   asm volatile(                                                                                        \
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"    \
@@ -203,6 +217,15 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),    \
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),   \
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]))
+
+// the same, from r[o .. o + 15] of a larger register array
+#define KVQ_ST16_AT(taddr, r, o)                                                                       \
+  asm volatile(                                                                                         \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"     \
+      "%15,%16};" ::"r"(taddr),                                                                         \
+      "r"(r[o + 0]), "r"(r[o + 1]), "r"(r[o + 2]), "r"(r[o + 3]), "r"(r[o + 4]), "r"(r[o + 5]),           \
+      "r"(r[o + 6]), "r"(r[o + 7]), "r"(r[o + 8]), "r"(r[o + 9]), "r"(r[o + 10]), "r"(r[o + 11]),         \
+      "r"(r[o + 12]), "r"(r[o + 13]), "r"(r[o + 14]), "r"(r[o + 15]))
 
 #define KVQ_ST16(taddr, r)                                                                              \
   asm volatile(                                                                                         \
@@ -250,28 +273,129 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 8 nibble codes of one word (feature e in bits 4e..4e+3) to the exact floats
-// code - 7.  Each nibble is masked into mantissa bits 12..15 or 16..19 of 1.0,
-// which makes 1 + n/2048 or 1 + n/128, and one FMA takes that to n - 7.
-__device__ __forceinline__ void nibbles_to_f32(uint32_t w, float (&v)[8]) {
-  const uint32_t a = w << 12, b = w << 4, c = w >> 8, d = w >> 12;
-  auto lo = [](uint32_t x) { return __uint_as_float(0x3F800000u | (x & 0x0000F000u)); };
-  auto hi = [](uint32_t x) { return __uint_as_float(0x3F800000u | (x & 0x000F0000u)); };
-  v[0] = fmaf(lo(a), 2048.f, -2055.f);
-  v[1] = fmaf(hi(a), 128.f, -135.f);
-  v[2] = fmaf(lo(b), 2048.f, -2055.f);
-  v[3] = fmaf(hi(b), 128.f, -135.f);
-  v[4] = fmaf(hi(w), 128.f, -135.f);
-  v[5] = fmaf(lo(c), 2048.f, -2055.f);
-  v[6] = fmaf(hi(c), 128.f, -135.f);
-  v[7] = fmaf(hi(d), 128.f, -135.f);
+// One K or V unit (a 128-token half-block of packed codes + scales in the
+// ring) to bf16 values (code - qmax) * scale in a swizzled 128 x 128 tile.
+// Warp wk converts tokens [32 wk, 32 wk + 32) -- for K that is one scale
+// group, whose 128 feature scales each lane loads once for its chunk.  Lanes
+// cover consecutive 16-byte code chunks, so the code reads are conflict-free.
+// The code - qmax step is exact in f32; the product with the f32 scale is
+// rounded once, to bf16.  Tokens at or past nv become zeros.
+
+// 4-bit: lane = 8 tokens x 4 chunks of 32 features; a byte's two nibbles go
+// into one f32x2 pair (nibble_pair), one FMA makes them n - 7 exactly.
+template <bool kV>
+__device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned char* dst, int wk, int lane, int nv) {
+  constexpr int kCb = 64;
+  const int q = lane & 3, tt = lane >> 2;
+  const float* sc = reinterpret_cast<const float*>(u + kBT * kCb);
+  u64 ks[16];
+  if (!kV) {
+    if (32 * wk < nv) {
+      const float4* s4 = reinterpret_cast<const float4*>(sc + wk * kD + 32 * q);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = s4[i];
+        ks[2 * i] = pack2(v.x, v.y);
+        ks[2 * i + 1] = pack2(v.z, v.w);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ks[i] = 0ull;
+    }
+  }
+  const u64 mul = pack2(256.f, 16.f), add = pack2(-263.f, -23.f);
+#pragma unroll 2
+  for (int it = 0; it < 4; ++it) {
+    const int t = 32 * wk + 8 * it + tt;
+    uint4 o[4];
+    if (t < nv) {
+      const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * kCb + 16 * q);
+      const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+      u64 s2 = 0ull;
+      if (kV) {
+        const float s = sc[4 * t + q];
+        s2 = pack2(s, s);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t h[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const u64 f = fma2(nibble_pair(byte_at15(w[i], r)), mul, add);
+          const u64 x = mul2(f, kV ? s2 : ks[4 * i + r]);
+          h[r] = pack_bf16(lo_f(x), hi_f(x));
+        }
+        o[i] = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int ch = 4 * q + i;
+      *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
+    }
+  }
 }
 
-// 4 byte codes of one word to the exact floats code - 127: the byte goes into
-// the low mantissa bits of 2^23 with one byte permute.
-__device__ __forceinline__ void bytes_to_f32(uint32_t w, float (&v)[4]) {
+// 8-bit: lane = 4 tokens x 8 chunks of 16 features; two bytes go into the
+// low mantissa bits of an f32x2 pair of 2^23, one add makes them c - 127.
+template <bool kV>
+__device__ __forceinline__ void decode_unit8(const unsigned char* u, unsigned char* dst, int wk, int lane, int nv) {
+  constexpr int kCb = 128;
+  const int q = lane & 7, tt = lane >> 3;
+  const float* sc = reinterpret_cast<const float*>(u + kBT * kCb);
+  u64 ks[8];
+  if (!kV) {
+    if (32 * wk < nv) {
+      const float4* s4 = reinterpret_cast<const float4*>(sc + wk * kD + 16 * q);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) v[k] = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + k)) - 8388735.f;
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = s4[i];
+        ks[2 * i] = pack2(v.x, v.y);
+        ks[2 * i + 1] = pack2(v.z, v.w);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ks[i] = 0ull;
+    }
+  }
+  const u64 sub = pack2(-8388735.f, -8388735.f);
+#pragma unroll 2
+  for (int it = 0; it < 8; ++it) {
+    const int t = 32 * wk + 4 * it + tt;
+    uint4 o[2];
+    if (t < nv) {
+      const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * kCb + 16 * q);
+      const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+      u64 s2 = 0ull;
+      if (kV) {
+        const float s = sc[4 * t + (q >> 1)];
+        s2 = pack2(s, s);
+      }
+      uint32_t h[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int r = 0; r < 4; r += 2) {
+          const u64 f = add2(byte_pair(w[i], r), sub);
+          const u64 x = mul2(f, kV ? s2 : ks[2 * i + r / 2]);
+          h[2 * i + r / 2] = pack_bf16(lo_f(x), hi_f(x));
+        }
+      }
+      o[0] = make_uint4(h[0], h[1], h[2], h[3]);
+      o[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    } else {
+      o[0] = make_uint4(0u, 0u, 0u, 0u);
+      o[1] = o[0];
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int ch = 2 * q + i;
+      *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -333,35 +457,37 @@ struct Cursor {
   __device__ __forceinline__ bool last() const { return j + 1 == seg.je; }
 };
 
-// Row maximum of one S tile row (128 columns in TMEM), scaled by qscale:
-// max over the valid columns of s * qscale, taken as max(sgn * s) * |qscale|.
-template <bool kNeg>
-__device__ __forceinline__ float row_max(uint32_t s_col, int nv, float aq) {
-  float mb = -INFINITY;
-#pragma unroll 1
-  for (int c = 0; c < 4; c += 2) {
-    uint32_t sa[32], sb[32];
-    KVQ_LD32(sa, s_col + 32u * c);
-    KVQ_LD32(sb, s_col + 32u * (c + 1));
-    tmem_wait_ld();
-    if (nv >= kBT) {
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Maximum (kMin: minimum) of 64 raw scores held in registers, as eight
+// independent three-input chains.
+template <bool kMin>
+__device__ __forceinline__ float row_extreme(const uint32_t (&sr)[64]) {
+  auto f = [](uint32_t x) { return __uint_as_float(x); };
+  auto op3 = [](float a, float b, float c) { return kMin ? min3(a, b, c) : max3(a, b, c); };
+  float acc[8];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float x = kNeg ? -__uint_as_float(sa[e]) : __uint_as_float(sa[e]);
-        const float y = kNeg ? -__uint_as_float(sb[e]) : __uint_as_float(sb[e]);
-        mb = fmaxf(mb, fmaxf(x, y));
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float x = kNeg ? -__uint_as_float(sa[e]) : __uint_as_float(sa[e]);
-        const float y = kNeg ? -__uint_as_float(sb[e]) : __uint_as_float(sb[e]);
-        if (32 * c + e < nv) mb = fmaxf(mb, x);
-        if (32 * (c + 1) + e < nv) mb = fmaxf(mb, y);
-      }
-    }
+  for (int j = 0; j < 8; ++j) {
+    acc[j] = op3(f(sr[j]), f(sr[8 + j]), f(sr[16 + j]));        // columns 0..23
+    acc[j] = op3(acc[j], f(sr[24 + j]), f(sr[32 + j]));         // 24..39
+    acc[j] = op3(acc[j], f(sr[40 + j]), f(sr[48 + j]));         // 40..55
   }
-  return mb * aq;
+  const float a = op3(acc[0], acc[1], acc[2]);
+  const float b = op3(acc[3], acc[4], acc[5]);
+  const float c = op3(acc[6], acc[7], a);
+  float r = op3(b, c, f(sr[56]));
+#pragma unroll
+  for (int j = 57; j < 64; j += 2) r = op3(r, f(sr[j]), f(sr[j + 1 < 64 ? j + 1 : j]));   // 56..63
+  return r;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ CUtensorMap qmap, ChunkParams p) {
@@ -556,10 +682,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
     } else if (warp >= 12) {
       // ======================= decode K/V to bf16 tiles =======================
       const int wk = warp - 12;                          // 32-token group of each unit
-      const uint32_t qmask = static_cast<uint32_t>(cb / 16 - 1);   // 16-byte chunks per token - 1
-      const int tsh = p.bits == 4 ? 2 : 3;               // lane = token * chunks + chunk
-      const int q = lane & qmask;
-      const int tt = lane >> tsh;
       Cursor kc, vc;
       kc.start(pre, p.B, H, cr);
       vc.start(pre, p.B, H, cr);
@@ -572,82 +694,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         const unsigned char* u = sm + kOffRing + slot * unit_bytes;
         unsigned char* dst = sm + (is_v ? kOffV : kOffK + (kb & 1u) * 2 * kTileHalf);
         const int nv = min(kBT, slen[c.seg.b] - c.j * kBT);
-        const bool gvalid = wk * 32 < nv;
         if (p.bits == 4) {
-          float ks[32];
-          if (!is_v && gvalid) {
-            const float4* s4 = reinterpret_cast<const float4*>(u + kBT * cb) + (wk * kD + 32 * q) / 4;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 v4 = s4[i];
-              ks[4 * i] = v4.x, ks[4 * i + 1] = v4.y, ks[4 * i + 2] = v4.z, ks[4 * i + 3] = v4.w;
-            }
-          }
-#pragma unroll 1
-          for (int it = 0; it < 4; ++it) {
-            const int t = 32 * wk + 8 * it + tt;
-            uint4 o[4] = {};
-            if (t < nv) {
-              const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * cb + 16 * q);
-              const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-              const float vs = is_v ? reinterpret_cast<const float*>(u + kBT * cb)[4 * t + q] : 0.f;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                float f[8];
-                nibbles_to_f32(w[i], f);
-                uint32_t h[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float s0 = is_v ? vs : ks[8 * i + 2 * e];
-                  const float s1 = is_v ? vs : ks[8 * i + 2 * e + 1];
-                  h[e] = pack_bf16(f[2 * e] * s0, f[2 * e + 1] * s1);
-                }
-                o[i] = make_uint4(h[0], h[1], h[2], h[3]);
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int ch = 4 * q + i;
-              *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
-            }
-          }
+          if (is_v) decode_unit4<true>(u, dst, wk, lane, nv);
+          else decode_unit4<false>(u, dst, wk, lane, nv);
         } else {
-          float ks[16];
-          if (!is_v && gvalid) {
-            const float4* s4 = reinterpret_cast<const float4*>(u + kBT * cb) + (wk * kD + 16 * q) / 4;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float4 v4 = s4[i];
-              ks[4 * i] = v4.x, ks[4 * i + 1] = v4.y, ks[4 * i + 2] = v4.z, ks[4 * i + 3] = v4.w;
-            }
-          }
-#pragma unroll 1
-          for (int it = 0; it < 8; ++it) {
-            const int t = 32 * wk + 4 * it + tt;
-            uint4 o[2] = {};
-            if (t < nv) {
-              const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * cb + 16 * q);
-              const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-              const float vs = is_v ? reinterpret_cast<const float*>(u + kBT * cb)[4 * t + (q >> 1)] : 0.f;
-              uint32_t h[8];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                float f[4];
-                bytes_to_f32(w[i], f);
-                const float s0 = is_v ? vs : ks[4 * i], s1 = is_v ? vs : ks[4 * i + 1];
-                const float s2 = is_v ? vs : ks[4 * i + 2], s3 = is_v ? vs : ks[4 * i + 3];
-                h[2 * i] = pack_bf16(f[0] * s0, f[1] * s1);
-                h[2 * i + 1] = pack_bf16(f[2] * s2, f[3] * s3);
-              }
-              o[0] = make_uint4(h[0], h[1], h[2], h[3]);
-              o[1] = make_uint4(h[4], h[5], h[6], h[7]);
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int ch = 2 * q + i;
-              *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
-            }
-          }
+          if (is_v) decode_unit8<true>(u, dst, wk, lane, nv);
+          else decode_unit8<false>(u, dst, wk, lane, nv);
         }
         fence_proxy_async();
         __syncwarp();
@@ -691,7 +743,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
           wait_bar(bar(S_FULL + tile), k & 1u, p.err, abort_flag);
           tc_fence_after();
           const int nv = min(kBT, slen[c.seg.b] - c.j * kBT);
-          const float mb = neg ? row_max<true>(s_col, nv, aq) : row_max<false>(s_col, nv, aq);
+          // pass 1: the row's extreme over the valid columns, 64 at a time
+          float mx = neg ? INFINITY : -INFINITY;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t sr[64];
+            KVQ_LD32_AT(sr, 0, s_col + 64u * hh);
+            KVQ_LD32_AT(sr, 32, s_col + 64u * hh + 32u);
+            tmem_wait_ld();
+            if (nv < kBT) {
+              // tokens past the sequence end stay out of the max
+              const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
+#pragma unroll
+              for (int e = 0; e < 64; ++e)
+                if (64 * hh + e >= nv) sr[e] = fill;
+            }
+            mx = neg ? fminf(mx, row_extreme<true>(sr)) : fmaxf(mx, row_extreme<false>(sr));
+          }
+          const float mb = mx * p.qscale;
           // lazy rescale: move the reference only when the block max outruns it
           const bool need = mb > m_ref + kLazy;
           const float m_new = need ? mb : m_ref;
@@ -709,42 +778,31 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
               KVQ_ST32(o_col + 32u * cc, orr);
             }
           }
-          // p = exp2(s * qscale - m_ref) as bf16, written over the S columns
-          const float nm = -m_ref;
+          // pass 2: p = exp2(s * qscale - m_ref) as bf16, written over the S columns
+          const u64 qs2 = pack2(p.qscale, p.qscale), nm2 = pack2(-m_ref, -m_ref);
+          u64 z2 = 0ull;
 #pragma unroll 1
-          for (int cc = 0; cc < 4; cc += 2) {
-            uint32_t sa[32], sb[32];
-            KVQ_LD32(sa, s_col + 32u * cc);
-            KVQ_LD32(sb, s_col + 32u * (cc + 1));
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t sr[64];
+            KVQ_LD32_AT(sr, 0, s_col + 64u * hh);
+            KVQ_LD32_AT(sr, 32, s_col + 64u * hh + 32u);
             tmem_wait_ld();
-            uint32_t pa[16], pb[16];
-            if (nv >= kBT) {
+            uint32_t pk[32];
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float p0 = ex2(fmaf(__uint_as_float(sa[2 * e]), p.qscale, nm));
-                const float p1 = ex2(fmaf(__uint_as_float(sa[2 * e + 1]), p.qscale, nm));
-                const float p2 = ex2(fmaf(__uint_as_float(sb[2 * e]), p.qscale, nm));
-                const float p3 = ex2(fmaf(__uint_as_float(sb[2 * e + 1]), p.qscale, nm));
-                z += (p0 + p1) + (p2 + p3);
-                pa[e] = pack_bf16(p0, p1);
-                pb[e] = pack_bf16(p2, p3);
+            for (int e = 0; e < 32; ++e) {
+              const u64 x = fma2(pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), qs2, nm2);
+              float p0 = ex2(lo_f(x)), p1 = ex2(hi_f(x));
+              if (nv < kBT) {
+                p0 = 64 * hh + 2 * e < nv ? p0 : 0.f;
+                p1 = 64 * hh + 2 * e + 1 < nv ? p1 : 0.f;
               }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int t0 = 32 * cc + 2 * e, t1 = t0 + 32;
-                const float p0 = t0 < nv ? ex2(fmaf(__uint_as_float(sa[2 * e]), p.qscale, nm)) : 0.f;
-                const float p1 = t0 + 1 < nv ? ex2(fmaf(__uint_as_float(sa[2 * e + 1]), p.qscale, nm)) : 0.f;
-                const float p2 = t1 < nv ? ex2(fmaf(__uint_as_float(sb[2 * e]), p.qscale, nm)) : 0.f;
-                const float p3 = t1 + 1 < nv ? ex2(fmaf(__uint_as_float(sb[2 * e + 1]), p.qscale, nm)) : 0.f;
-                z += (p0 + p1) + (p2 + p3);
-                pa[e] = pack_bf16(p0, p1);
-                pb[e] = pack_bf16(p2, p3);
-              }
+              z2 = add2(z2, pack2(p0, p1));
+              pk[e] = pack_bf16(p0, p1);
             }
-            KVQ_ST16(s_col + 16u * cc, pa);
-            KVQ_ST16(s_col + 16u * (cc + 1), pb);
+            KVQ_ST16_AT(s_col + 32u * hh, pk, 0);
+            KVQ_ST16_AT(s_col + 32u * hh + 16u, pk, 16);
           }
+          z += lo_f(z2) + hi_f(z2);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();

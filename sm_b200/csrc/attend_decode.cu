@@ -40,13 +40,12 @@
 // sum q'' f - sum q'' (1 + 7 eps) = sum q' (n - 7): the second sum is one
 // correction per block.  For V, u = (U - (1 + 7 eps) P) / eps with U = sum p' f
 // and P = sum p'.  Rounding error is amplified by at most 2^8 / 7.
+#include "f32x2.cuh"
 #include "kvq_internal.cuh"
 #include "plan.cuh"
 
 namespace kvq {
 namespace {
-
-typedef unsigned long long u64;       // one f32x2 value (low half = first float)
 
 constexpr int kD = 128;
 constexpr int kG = 4;                 // query heads per KV head
@@ -196,51 +195,13 @@ __device__ __forceinline__ float warp_max(float v) {
   return r;
 }
 
-// f32x2 values travel in 64-bit registers from the instruction that makes
-// them to the instruction that uses them, so no register-pair moves are
-// needed around the packed FMAs (u64 is declared with the constants).
-
-__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
-  u64 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
-__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
-  u64 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-__device__ __forceinline__ u64 pack2(float lo, float hi) {
-  u64 d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-
-__device__ __forceinline__ float lo_f(u64 x) { return __uint_as_float(static_cast<uint32_t>(x)); }
-__device__ __forceinline__ float hi_f(u64 x) { return __uint_as_float(static_cast<uint32_t>(x >> 32)); }
-
-// The two channels of one code byte after a shift that puts them at bits
-// 15..18 and 19..22: (1 + n_even 2^-8, 1 + n_odd 2^-4) as one f32x2 value.
-__device__ __forceinline__ u64 nibble_pair(uint32_t a) {
-  u64 x;
-  asm("{.reg .b32 t0, t1;\n\t"
-      "lop3.b32 t0, %1, 0x00078000, 0x3F800000, 0xEA;\n\t"
-      "lop3.b32 t1, %1, 0x00780000, 0x3F800000, 0xEA;\n\t"
-      "mov.b64 %0, {t0, t1};}"
-      : "=l"(x)
-      : "r"(a));
-  return x;
-}
-
 // Channel pairs (16cs + 2i, 16cs + 2i + 1), i = 0..7, of one 64-bit code load.
 __device__ __forceinline__ void nibble_pairs(uint32_t w0, uint32_t w1, u64 f[8]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t w = i < 4 ? w0 : w1;
     const int r = i & 3;
-    f[i] = nibble_pair(r == 0 ? (w << 15) : r == 1 ? (w << 7) : r == 2 ? (w >> 1) : (w >> 9));
+    f[i] = nibble_pair(byte_at15(w, r));
   }
 }
 

@@ -9,9 +9,8 @@
 // Two layouts of the per-CTA partial states.  Row-major ([slot][row][m, z,
 // u...]), for the few-row decode kernels: one CTA per (b, h), a warp per row.
 // Feature-major ([slot][field][row]), for the many-row chunk kernel: one CTA
-// per (b, h) and 32-row chunk, lane = row so every partial read is a
-// coalesced 128-byte line, the merged tile staged in shared memory and
-// written out as whole rows.
+// per (b, h), 32-row chunk and 32-feature slice, lane = row so every partial
+// read is a coalesced 128-byte line.
 //
 // A (b, h) that one CTA covered whole was already written by that CTA and is
 // skipped here.  The merge also owns the sequences with no valid key: it
@@ -75,82 +74,104 @@ __global__ void __launch_bounds__(128) merge_kernel(MergeParams mp) {
 }
 
 constexpr int kFmRows = 32;       // rows per CTA of the feature-major merge
-constexpr int kFmThreads = 256;
+constexpr int kFmCols = 32;       // features per CTA
+constexpr int kFmThreads = 128;   // 4 warps x 8 features
+constexpr int kFmBatch = 4;       // parts whose weights are held at once
 
-__global__ void __launch_bounds__(kFmThreads) merge_fm_kernel(MergeParams mp) {
-  extern __shared__ float s_tile[];                // [kFmRows][D + 1], then int pre[B + 1]
+// Feature-major merge: one CTA per (b, h), 32-row chunk and 32-feature
+// slice; lane = row, so every read of a part's field is one coalesced
+// 128-byte line; warp w owns 8 features.  The weights exp(m_c - m) of up to
+// four parts sit in registers and each part's 8 values are loaded together.
+__global__ void __launch_bounds__(kFmThreads, 4) merge_fm_kernel(MergeParams mp) {
+  extern __shared__ int s_pre[];                   // [B + 1]
   const MergeArgs& a = mp.a;
   const int D = a.D;
-  int* s_pre = reinterpret_cast<int*>(s_tile + kFmRows * (D + 1));
   if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
   __syncthreads();
   const int H = a.H_kv;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
-  const int r0 = blockIdx.y * kFmRows;
-  const int rows = min(kFmRows, a.R - r0);
-  const long long row_base = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = blockIdx.y * kFmRows + lane;
+  const int f0 = blockIdx.z * kFmCols + 8 * warp;
+  const long long row = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r;
   const int raw_len = a.lengths[b];
-  if (h == 0 && blockIdx.y == 0 && threadIdx.x == 0 && (raw_len < 1 || raw_len > a.N_cap))
+  if (h == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0 && (raw_len < 1 || raw_len > a.N_cap))
     record_error(mp.err, KVQ_ERR_LENGTH);
+  const bool live = r < a.R && f0 < D;
   const int nb = s_pre[b + 1] - s_pre[b];
   if (nb == 0) {
-    for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x)
-      store_from_f32(a.O, row_base * D + idx, 0.f, a.o_dtype);
+    if (live)
+      for (int j = 0; j < 8 && f0 + j < D; ++j) store_from_f32(a.O, row * D + f0 + j, 0.f, a.o_dtype);
     return;
   }
   const CtaRange cr = cta_range(s_pre, a.B, H, a.ctas, 0);
   const long long S = static_cast<long long>(H) * s_pre[b] + static_cast<long long>(h) * nb;
   const long long E = S + nb;
   const long long c_first = S / cr.P, c_last = (E - 1) / cr.P;
-  if (c_first == c_last) return;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  if (c_first == c_last || !live) return;
   const long long slot_floats = static_cast<long long>(D + 2) * a.R_pad;
-  if (lane < rows) {
-    const int r = r0 + lane;
-    float m = -INFINITY;
-    for (long long c = c_first; c <= c_last; ++c) {
-      const float* part = a.partials + (c + bh) * slot_floats + r;
-      if (part[a.R_pad] > 0.f) m = fmaxf(m, part[0]);
-    }
-    float z = 0.f;
-    for (long long c = c_first; c <= c_last; ++c) {
-      const float* part = a.partials + (c + bh) * slot_floats + r;
-      const float zc = part[a.R_pad];
-      if (zc > 0.f) z += expf(part[0] - m) * zc;
-    }
-    const float inv = 1.f / z;
-    for (int d = warp; d < D; d += nwarps) {
-      float u = 0.f;
-      for (long long c = c_first; c <= c_last; ++c) {
-        const float* part = a.partials + (c + bh) * slot_floats + r;
-        const float zc = part[a.R_pad];
-        if (zc > 0.f) u += expf(part[0] - m) * part[static_cast<long long>(2 + d) * a.R_pad];
-      }
-      s_tile[lane * (D + 1) + d] = u * inv;
-    }
+  const long long rp = a.R_pad;
+  const float* col = a.partials + bh * slot_floats + r;       // part c of this row: col + c * slot_floats
+  float m = -INFINITY;
+#pragma unroll 4
+  for (long long c = c_first; c <= c_last; ++c) {
+    const float* part = col + c * slot_floats;
+    const float zc = part[rp], mc = part[0];
+    if (zc > 0.f) m = fmaxf(m, mc);
   }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x)
-    store_from_f32(a.O, row_base * D + idx, s_tile[(idx / D) * (D + 1) + idx % D], a.o_dtype);
+  float z = 0.f, u[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) u[j] = 0.f;
+  const int nf = min(8, D - f0);
+  for (long long cb = c_first; cb <= c_last; cb += kFmBatch) {
+    float wgt[kFmBatch], v[kFmBatch][8];
+#pragma unroll
+    for (int k = 0; k < kFmBatch; ++k) {
+      const long long c = min(cb + k, c_last);
+      const float* part = col + c * slot_floats;
+      const float zc = part[rp], mc = part[0];
+      wgt[k] = (cb + k <= c_last && zc > 0.f) ? expf(mc - m) : 0.f;
+      z += wgt[k] * (zc > 0.f ? zc : 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[k][j] = j < nf ? part[(2 + f0 + j) * rp] : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kFmBatch; ++k)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u[j] = fmaf(wgt[k], v[k][j], u[j]);
+  }
+  const float inv = 1.f / z;
+  if (a.o_dtype == KVQ_BF16 && nf == 8) {
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 t = __floats2bfloat162_rn(u[2 * j] * inv, u[2 * j + 1] * inv);
+      o[j] = *reinterpret_cast<const uint32_t*>(&t);
+    }
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + row * D + f0) = make_uint4(o[0], o[1], o[2], o[3]);
+  } else {
+    for (int j = 0; j < nf; ++j) store_from_f32(a.O, row * D + f0 + j, u[j] * inv, a.o_dtype);
+  }
 }
 
 }  // namespace
 
 kvq_status launch_merge(const MergeArgs& a, cudaStream_t s) {
   if (a.feature_major) {
-    const size_t smem = static_cast<size_t>(kFmRows) * (a.D + 1) * sizeof(float) +
-                        static_cast<size_t>(a.B + 1) * sizeof(int);
+    const size_t smem = static_cast<size_t>(a.B + 1) * sizeof(int);
     const long long bh = static_cast<long long>(a.B) * a.H_kv;
     const int chunks = (a.R + kFmRows - 1) / kFmRows;
-    if (bh > 0x7fffffffLL || chunks > 65535) return KVQ_ERR_UNSUPPORTED;
+    const int slices = (a.D + kFmCols - 1) / kFmCols;
+    if (bh > 0x7fffffffLL || chunks > 65535 || slices > 65535 || (a.D % 8) != 0) return KVQ_ERR_UNSUPPORTED;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(merge_fm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return KVQ_ERR_UNSUPPORTED;
     MergeParams mp{a, error_word()};
     if (!mp.err) return KVQ_ERR_CUDA;
-    merge_fm_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(chunks)), kFmThreads, smem, s>>>(mp);
+    merge_fm_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(chunks), static_cast<unsigned>(slices)),
+                      kFmThreads, smem, s>>>(mp);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
   }
