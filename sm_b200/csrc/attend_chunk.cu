@@ -52,9 +52,12 @@
 #include "f32x2.cuh"
 #include "kvq_internal.cuh"
 #include "plan.cuh"
+#include "tc_common.cuh"
 
 namespace kvq {
 namespace {
+
+using namespace tc;
 
 constexpr int kD = 128;
 constexpr int kBT = 128;              // tokens per block
@@ -108,171 +111,6 @@ struct ChunkParams {
 
 size_t smem_bytes(int B) { return 1024 + kOffPre + sizeof(int) * (2 * B + 1); }
 
-// ---------------------------------------------------------------------------
-// PTX helpers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t su(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(100000u)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait: after about two seconds record KVQ_ERR_TIMEOUT, raise the
-// CTA's abort flag and go on; once the flag is up every later wait of the CTA
-// returns at once, so the kernel always reaches its end (and frees its tensor
-// memory) within a few seconds.
-__device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, unsigned int* err, volatile int* abort_flag) {
-  if (mbar_try(bar, parity)) return;
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try(bar, parity)) {
-    if (*abort_flag) return;
-    if (globaltimer() - t0 > 2000000000ull) {
-      record_error(err, KVQ_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return;
-    }
-  }
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(
-          d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-
-#define KVQ_LD32(r, taddr)                                                                             \
-  asm volatile(                                                                                        \
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"  \
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                        \
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),        \
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),      \
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),      \
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                           \
-      : "r"(taddr))
-
-// the same, into r[o .. o + 31] of a larger register array
-#define KVQ_LD32_AT(r, o, taddr)                                                                       \
-  asm volatile(                                                                                        \
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"  \
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                        \
-      : "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]),   \
-        "=r"(r[o + 6]), "=r"(r[o + 7]), "=r"(r[o + 8]), "=r"(r[o + 9]), "=r"(r[o + 10]), "=r"(r[o + 11]), \
-        "=r"(r[o + 12]), "=r"(r[o + 13]), "=r"(r[o + 14]), "=r"(r[o + 15]), "=r"(r[o + 16]),             \
-        "=r"(r[o + 17]), "=r"(r[o + 18]), "=r"(r[o + 19]), "=r"(r[o + 20]), "=r"(r[o + 21]),             \
-        "=r"(r[o + 22]), "=r"(r[o + 23]), "=r"(r[o + 24]), "=r"(r[o + 25]), "=r"(r[o + 26]),             \
-        "=r"(r[o + 27]), "=r"(r[o + 28]), "=r"(r[o + 29]), "=r"(r[o + 30]), "=r"(r[o + 31])              \
-      : "r"(taddr))
-
-#define KVQ_ST32(taddr, r)                                                                             \
-  asm volatile(                                                                                        \
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"    \
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),          \
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), \
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),    \
-      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),   \
-      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]))
-
-// the same, from r[o .. o + 15] of a larger register array
-#define KVQ_ST16_AT(taddr, r, o)                                                                       \
-  asm volatile(                                                                                         \
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"     \
-      "%15,%16};" ::"r"(taddr),                                                                         \
-      "r"(r[o + 0]), "r"(r[o + 1]), "r"(r[o + 2]), "r"(r[o + 3]), "r"(r[o + 4]), "r"(r[o + 5]),           \
-      "r"(r[o + 6]), "r"(r[o + 7]), "r"(r[o + 8]), "r"(r[o + 9]), "r"(r[o + 10]), "r"(r[o + 11]),         \
-      "r"(r[o + 12]), "r"(r[o + 13]), "r"(r[o + 14]), "r"(r[o + 15]))
-
-#define KVQ_ST16(taddr, r)                                                                              \
-  asm volatile(                                                                                         \
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"     \
-      "%15,%16};" ::"r"(taddr),                                                                         \
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),  \
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]))
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// UMMA shared-memory descriptor: 128-byte swizzle, 1 KB eight-row atoms.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
-         (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor, kind::f16: bf16 A and B, f32 accumulate, M = 128.
-__host__ __device__ constexpr uint32_t instr_desc(int n, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) |
-         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
-}
-
-// Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a swizzled 64-wide half.
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-  return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
 // One K or V unit (a 128-token half-block of packed codes + scales in the
 // ring) to bf16 values (code - qmax) * scale in a swizzled 128 x 128 tile.
 // Warp wk converts tokens [32 wk, 32 wk + 32) -- for K that is one scale
@@ -282,21 +120,28 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 // rounded once, to bf16.  Tokens at or past nv become zeros.
 
 // 4-bit: lane = 8 tokens x 4 chunks of 32 features; a byte's two nibbles go
-// into one f32x2 pair (nibble_pair), one FMA makes them n - 7 exactly.
+// into one f32x2 pair (nibble_pair), one FMA makes them n - 7 exactly.  Lane
+// q handles its four words in the order q, q + 1, ... (mod 4): the eight lanes
+// of a quarter warp then store to eight different bank groups, and the K
+// scale loads of a quarter warp hit four groups (lanes of one q share an
+// address).
 template <bool kV>
 __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned char* dst, int wk, int lane, int nv) {
   constexpr int kCb = 64;
   const int q = lane & 3, tt = lane >> 2;
   const float* sc = reinterpret_cast<const float*>(u + kBT * kCb);
-  u64 ks[16];
+  u64 ks[16];                                   // slot 4 i + r: pair r of word (i + q) mod 4
   if (!kV) {
     if (32 * wk < nv) {
       const float4* s4 = reinterpret_cast<const float4*>(sc + wk * kD + 32 * q);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 v = s4[i];
-        ks[2 * i] = pack2(v.x, v.y);
-        ks[2 * i + 1] = pack2(v.z, v.w);
+      for (int i = 0; i < 4; ++i) {
+        const int wi = (i + q) & 3;
+        const float4 v0 = s4[2 * wi], v1 = s4[2 * wi + 1];
+        ks[4 * i] = pack2(v0.x, v0.y);
+        ks[4 * i + 1] = pack2(v0.z, v0.w);
+        ks[4 * i + 2] = pack2(v1.x, v1.y);
+        ks[4 * i + 3] = pack2(v1.z, v1.w);
       }
     } else {
 #pragma unroll
@@ -310,7 +155,18 @@ __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned ch
     uint4 o[4];
     if (t < nv) {
       const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * kCb + 16 * q);
-      const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+      // w[i] = word (i + q) mod 4
+      uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+      {
+        const bool c = (q & 2) != 0;
+        const uint32_t x0 = c ? w[2] : w[0], x1 = c ? w[3] : w[1], x2 = c ? w[0] : w[2], x3 = c ? w[1] : w[3];
+        w[0] = x0, w[1] = x1, w[2] = x2, w[3] = x3;
+      }
+      {
+        const bool c = (q & 1) != 0;
+        const uint32_t x0 = c ? w[1] : w[0], x1 = c ? w[2] : w[1], x2 = c ? w[3] : w[2], x3 = c ? w[0] : w[3];
+        w[0] = x0, w[1] = x1, w[2] = x2, w[3] = x3;
+      }
       u64 s2 = 0ull;
       if (kV) {
         const float s = sc[4 * t + q];
@@ -333,7 +189,7 @@ __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned ch
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int ch = 4 * q + i;
+      const int ch = 4 * q + ((i + q) & 3);
       *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
     }
   }
@@ -341,20 +197,26 @@ __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned ch
 
 // 8-bit: lane = 4 tokens x 8 chunks of 16 features; two bytes go into the
 // low mantissa bits of an f32x2 pair of 2^23, one add makes them c - 127.
+// Lanes q and q + 4 store their two 16-byte chunks in opposite order, so a
+// quarter warp (one token) stores to eight different bank groups.
 template <bool kV>
 __device__ __forceinline__ void decode_unit8(const unsigned char* u, unsigned char* dst, int wk, int lane, int nv) {
   constexpr int kCb = 128;
   const int q = lane & 7, tt = lane >> 3;
+  const bool swap = (q & 4) != 0;
   const float* sc = reinterpret_cast<const float*>(u + kBT * kCb);
-  u64 ks[8];
+  u64 ks[8];                                    // slot 4 i + r: pair r of chunk i ^ swap
   if (!kV) {
     if (32 * wk < nv) {
       const float4* s4 = reinterpret_cast<const float4*>(sc + wk * kD + 16 * q);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = s4[i];
-        ks[2 * i] = pack2(v.x, v.y);
-        ks[2 * i + 1] = pack2(v.z, v.w);
+      for (int i = 0; i < 2; ++i) {
+        const int ci = i ^ (swap ? 1 : 0);
+        const float4 v0 = s4[2 * ci], v1 = s4[2 * ci + 1];
+        ks[4 * i] = pack2(v0.x, v0.y);
+        ks[4 * i + 1] = pack2(v0.z, v0.w);
+        ks[4 * i + 2] = pack2(v1.x, v1.y);
+        ks[4 * i + 3] = pack2(v1.z, v1.w);
       }
     } else {
 #pragma unroll
@@ -368,7 +230,7 @@ __device__ __forceinline__ void decode_unit8(const unsigned char* u, unsigned ch
     uint4 o[2];
     if (t < nv) {
       const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * kCb + 16 * q);
-      const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+      const uint32_t w[4] = {swap ? w4.z : w4.x, swap ? w4.w : w4.y, swap ? w4.x : w4.z, swap ? w4.y : w4.w};
       u64 s2 = 0ull;
       if (kV) {
         const float s = sc[4 * t + (q >> 1)];
@@ -392,80 +254,10 @@ __device__ __forceinline__ void decode_unit8(const unsigned char* u, unsigned ch
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const int ch = 2 * q + i;
+      const int ch = 2 * q + (i ^ (swap ? 1 : 0));
       *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
     }
   }
-}
-
-// ---------------------------------------------------------------------------
-// the CTA's blocks, one at a time (same walk as the plan)
-// ---------------------------------------------------------------------------
-struct Seg {
-  int b, h, nb, jb, je;
-  long long gpos;
-  bool valid;
-};
-__device__ __forceinline__ Seg first_seg(const int* pre, int B, int H, const CtaRange& cr) {
-  Seg s;
-  s.valid = cr.g0 < cr.g1;
-  if (!s.valid) return s;
-  s.b = find_seq(pre, B, H, cr.g0);
-  s.nb = pre[s.b + 1] - pre[s.b];
-  const long long off = cr.g0 - static_cast<long long>(H) * pre[s.b];
-  s.h = static_cast<int>(off / s.nb);
-  s.jb = static_cast<int>(off % s.nb);
-  s.je = static_cast<int>(min(static_cast<long long>(s.nb), s.jb + (cr.g1 - cr.g0)));
-  s.gpos = cr.g0;
-  return s;
-}
-__device__ __forceinline__ Seg next_seg(Seg s, const int* pre, int B, int H, const CtaRange& cr) {
-  s.gpos += s.je - s.jb;
-  if (s.gpos >= cr.g1) {
-    s.valid = false;
-    return s;
-  }
-  if (++s.h == H) {
-    s.h = 0;
-    ++s.b;
-    while (s.b < B && pre[s.b + 1] == pre[s.b]) ++s.b;
-  }
-  s.nb = pre[s.b + 1] - pre[s.b];
-  s.jb = 0;
-  s.je = static_cast<int>(min(static_cast<long long>(s.nb), cr.g1 - s.gpos));
-  return s;
-}
-
-// A position in the CTA's block list: segment (one (b, h)) and block j in it.
-struct Cursor {
-  Seg seg;
-  int j;
-  bool valid;
-  __device__ __forceinline__ void start(const int* pre, int B, int H, const CtaRange& cr) {
-    seg = first_seg(pre, B, H, cr);
-    j = seg.jb;
-    valid = seg.valid && seg.jb < seg.je;
-  }
-  __device__ __forceinline__ void next(const int* pre, int B, int H, const CtaRange& cr) {
-    if (++j == seg.je) {
-      seg = next_seg(seg, pre, B, H, cr);
-      j = seg.jb;
-      valid = seg.valid;
-    }
-  }
-  __device__ __forceinline__ bool first() const { return j == seg.jb; }
-  __device__ __forceinline__ bool last() const { return j + 1 == seg.je; }
-};
-
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-__device__ __forceinline__ float min3(float a, float b, float c) {
-  float r;
-  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
 }
 
 // Maximum (kMin: minimum) of 64 raw scores held in registers, as eight

@@ -211,6 +211,45 @@ def test_chunk_tensor_core_ragged(sm, bits, lq):
         _check_gqa(sm, q, k, v, lens, bits, 32, 1.0, splits=splits)
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("hq,hkv,lq", [(8, 2, 1), (4, 2, 1), (2, 2, 1), (2, 2, 3), (4, 2, 2)])
+def test_decode_rows(sm, bits, hq, hkv, lq):
+    """One to four query rows per KV head at D = 128, g = 32: lengths that end
+    inside a block and inside a K group, one a power of two, one shorter
+    than a K group, and several splits."""
+    q, k, v, lens = _gqa_case(4, hq, hkv, 700, 128, [700, 300, 128, 29], lq=lq, seed=31 + bits + hq + lq,
+                              bits=bits, outliers=True)
+    for splits in (0, 1, 5):
+        _check_gqa(sm, q, k, v, lens, bits, 32, 1.0, splits=splits)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_decode_fp32_q_sharp(sm, bits):
+    """f32 Q and a large score scale: the running maximum moves by far more
+    than any rescale threshold from block to block, and the softmax is far
+    from uniform."""
+    q, k, v, lens = _gqa_case(2, 8, 2, 1000, 128, [1000, 517], seed=40 + bits, bits=bits)
+    for j, f in enumerate([1.0, 2.0, 3.5, 5.0]):
+        k[:, :, 250 * j:250 * (j + 1), :] *= f      # keys grow along the sequence
+    k[:, :, ::128, :] *= 2.0                        # and one strong key per block
+    _check_gqa(sm, q, k, v, lens, bits, 32, 3.0, q_dtype=torch.float32, splits=3)
+
+
+def test_decode_bad_lengths(sm):
+    q, k, v, _ = _gqa_case(3, 8, 2, 256, 128, [256, 256, 256], seed=9)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    assert sm.kernel_name(cache, 8, 1).startswith("decode_gqa4")
+    out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+    lens = torch.tensor([256, 0, 200], dtype=torch.int32, device=DEV)
+    sm.attend(to_dev(q, torch.bfloat16), cache, lens, 1.0, out=out, splits=4)
+    with pytest.raises(sm.KVQError) as e:
+        sm.check()
+    assert e.value.name == "KVQ_ERR_LENGTH"
+    assert torch.all(out[1] == 0)
+    assert torch.isfinite(out.float()).all()
+    sm.check()
+
+
 def test_repeat_is_bit_identical(sm):
     q, k, v, lens = _gqa_case(2, 8, 2, 300, 128, [300, 200], seed=6)
     cache = pack_gpu(sm, k, v, 4, 32)
