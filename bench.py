@@ -50,6 +50,32 @@ SEED = 0
 
 
 # ---------------------------------------------------------------------------
+# ranks: the batch is sharded, one independent batch per rank (no collective
+# on the data path); the timing is the max over ranks
+# ---------------------------------------------------------------------------
+
+def rank_seed(rank: int) -> int:
+    """Seed of rank `rank`'s batch: every rank attends its own sequences."""
+    return SEED + rank
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max over the ranks of a list of floats (all_reduce MAX of
+    the process group in use: NCCL on GPUs, gloo on CPU)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # byte accounting
 # ---------------------------------------------------------------------------
 
@@ -247,7 +273,7 @@ def run_kvq(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     workload = args.workload
-    q_np, k_np, v_np, lens_np, meta = W.gqa_case(workload, SEED + rank)
+    q_np, k_np, v_np, lens_np, meta = W.gqa_case(workload, rank_seed(rank))
     q_np = torch.from_numpy(q_np).to(torch.bfloat16).float().numpy()
     B, H_q, H_kv, D, N, Lq = meta["B"], meta["H_q"], meta["H_kv"], meta["D"], meta["N"], meta["Lq"]
     bits = args.bits if args.bits else (meta["bits"] if isinstance(meta["bits"], int) else 4)
@@ -375,16 +401,13 @@ def run_kvq(args, rank, world, local_rank):
     abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g, lq=Lq)
     step_bytes = abytes + (append_bytes(B, H_kv, D, N - t0, Lq, bits, g) if uniform else 0)
     attend_flops = 4 * H_q * Lq * D * int(np.sum(lens_np.astype(np.int64)))
-    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max, e2e_max = float(t[0]), float(t[1])
+    ms_max, e2e_max = max_over_ranks([ms, e2e_ms], world, dev)
 
     res = None
     if rank == 0:
         per_step_ms = ms_max / args.steps
-        value = world * step_bytes / (per_step_ms * 1e-3) / 1e9
-        e2e_value = world * step_bytes / (e2e_max / args.steps * 1e-3) / 1e9
+        value = whole_job_rate(step_bytes, world, per_step_ms) / 1e9
+        e2e_value = whole_job_rate(step_bytes, world, e2e_max / args.steps) / 1e9
         att_ms = statistics.mean(attend_ms)
         tensor = workload == "chunk"
         if tensor:
