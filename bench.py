@@ -175,16 +175,19 @@ class ClockSampler:
         except Exception as e:  # no NVML: clocks reported as unavailable
             self.err = str(e)
 
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self.period)
 
     def __enter__(self):
@@ -194,9 +197,12 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        # the region may be shorter than one polling period: one more sample
+        # at its end (the caller exits right after its end-of-region sync)
         if self.ok:
             self._stop.set()
             self.t.join()
+            self._sample()
 
     def summary(self):
         if not self.ok or not self.samples:
@@ -244,7 +250,11 @@ def oracle_step_sample(heads, q, k, v, lengths, meta, prepacked):
     return nbytes
 
 
-def cpu_oracle_rate(q, k, v, lengths, meta, n_heads: int, repeats: int = 1):
+def cpu_oracle_rate(q, k, v, lengths, meta, n_heads: int, repeats: int = 1, min_seconds: float = 0.0,
+                    max_repeats: int = 30):
+    """Bytes and per-pass seconds of the oracle over a sample of n_heads
+    (b, h_kv) heads: `repeats` passes, more (up to max_repeats) until the
+    passes add up to min_seconds."""
     import oracle as O
     rng = np.random.default_rng(123)
     all_heads = [(b, h) for b in range(meta["B"]) for h in range(meta["H_kv"])]
@@ -254,7 +264,7 @@ def cpu_oracle_rate(q, k, v, lengths, meta, n_heads: int, repeats: int = 1):
                     O.pack_v(v[b, h], meta["bits"], meta["group"])) for (b, h) in heads}
     times, nbytes = [], 0
     oracle_step_sample(heads[:1], q, k, v, lengths, meta, pre)   # warm
-    for _ in range(repeats):
+    while len(times) < repeats or (sum(times) < min_seconds and len(times) < max_repeats):
         t = time.perf_counter()
         nbytes = oracle_step_sample(heads, q, k, v, lengths, meta, pre)
         times.append(time.perf_counter() - t)
@@ -463,7 +473,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-heads", type=int, default=64,
+    ap.add_argument("--cpu-heads", type=int, default=256,
                     help="(b, h_kv) heads in the oracle's timed sample")
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD,
                     help="the decode GQA workload is the headline; the others are for study")
@@ -524,12 +534,14 @@ def main():
     res, data = run_kvq(args, rank, world, local_rank)
     if rank == 0 and not args.no_cpu_baseline:
         q, k, v, lens, meta = data
-        nb, ts, heads = cpu_oracle_rate(q, k, v, lens, meta, args.cpu_heads, repeats=3)
+        nb, ts, heads = cpu_oracle_rate(q, k, v, lens, meta, args.cpu_heads, repeats=3, min_seconds=10.0)
         rate = nb / statistics.median(ts) / 1e9
         res["cpu_baseline"] = {"value": round(rate, 4), "unit": "GB/s", "cores": blas_threads(),
                                "kind": "oracle",
-                               "sample": f"{len(heads)} of {meta['B'] * meta['H_kv']} (b, h_kv) heads, "
-                                         f"median of 3 passes ({statistics.median(ts):.2f} s each)"}
+                               "sample": f"{len(heads)} of {meta['B'] * meta['H_kv']} (b, h_kv) heads per pass "
+                                         f"(the append + attend of the step for those heads), median of "
+                                         f"{len(ts)} passes ({statistics.median(ts):.2f} s each, "
+                                         f"{sum(ts):.1f} s in all)"}
     if rank == 0:
         print(json.dumps(res))
     if world > 1:
