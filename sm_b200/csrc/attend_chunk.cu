@@ -19,7 +19,7 @@
 // the true running maximum gives the same u / z in exact arithmetic, and the
 // exponentials stay <= 2^8, well inside bf16/fp32 range.
 //
-// Warp roles (16 warps):
+// Warp roles (20 warps, 96 registers each):
 //   0        producer: cp.async.bulk of the packed codes + scales, one unit
 //            per K or V half of a block, into a ring of 54 KB (5 units at
 //            4 bits, 3 at 8 bits).  Unit order K(0), K(1), V(0), K(2), V(1),
@@ -29,7 +29,7 @@
 //            Q rows, once the previous segment's Q K^T products are done
 //   4..7     softmax of query rows 0..127 (TMEM lanes 0..127, warp w owns
 //            lanes 32*(w%4)..+31); 8..11 the same for rows 128..255
-//   12..15   decode: warp w converts the 32-token group w-12 of each K unit
+//   12..19   decode: warp w converts the 16-token slice w-12 of each K unit
 //            (into one of two K tiles) and the same tokens of each V unit
 //   3        idle
 // The MMA order per block k is QK0(k) QK1(k) | PV0(k) QK0(k+1) PV1(k)
@@ -61,7 +61,7 @@ using namespace tc;
 
 constexpr int kD = 128;
 constexpr int kBT = 128;              // tokens per block
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLazy = 8.f;          // log2 units a row max may outrun its reference
@@ -92,7 +92,7 @@ enum Bar {
   P_FULL = 20,                   // [2]
   PV_DONE = 22,                  // [2]
 };
-constexpr int kDecodeWarps = 4;
+constexpr int kDecodeWarps = 8;
 
 struct ChunkParams {
   const uint8_t* k_codes;
@@ -113,8 +113,8 @@ size_t smem_bytes(int B) { return 1024 + kOffPre + sizeof(int) * (2 * B + 1); }
 
 // One K or V unit (a 128-token half-block of packed codes + scales in the
 // ring) to bf16 values (code - qmax) * scale in a swizzled 128 x 128 tile.
-// Warp wk converts tokens [32 wk, 32 wk + 32) -- for K that is one scale
-// group, whose 128 feature scales each lane loads once for its chunk.  Lanes
+// Warp wk converts tokens [16 wk, 16 wk + 16) -- for K half of scale group
+// wk / 2, whose feature scales each lane loads once for its chunk.  Lanes
 // cover consecutive 16-byte code chunks, so the code reads are conflict-free.
 // The code - qmax step is exact in f32; the product with the f32 scale is
 // rounded once, to bf16.  Tokens at or past nv become zeros.
@@ -132,8 +132,8 @@ __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned ch
   const float* sc = reinterpret_cast<const float*>(u + kBT * kCb);
   u64 ks[16];                                   // slot 4 i + r: pair r of word (i + q) mod 4
   if (!kV) {
-    if (32 * wk < nv) {
-      const float4* s4 = reinterpret_cast<const float4*>(sc + wk * kD + 32 * q);
+    if (16 * wk < nv) {
+      const float4* s4 = reinterpret_cast<const float4*>(sc + (wk >> 1) * kD + 32 * q);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int wi = (i + q) & 3;
@@ -149,9 +149,9 @@ __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned ch
     }
   }
   const u64 mul = pack2(256.f, 16.f), add = pack2(-263.f, -23.f);
-#pragma unroll 2
-  for (int it = 0; it < 4; ++it) {
-    const int t = 32 * wk + 8 * it + tt;
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int t = 16 * wk + 8 * it + tt;
     uint4 o[4];
     if (t < nv) {
       const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * kCb + 16 * q);
@@ -207,8 +207,8 @@ __device__ __forceinline__ void decode_unit8(const unsigned char* u, unsigned ch
   const float* sc = reinterpret_cast<const float*>(u + kBT * kCb);
   u64 ks[8];                                    // slot 4 i + r: pair r of chunk i ^ swap
   if (!kV) {
-    if (32 * wk < nv) {
-      const float4* s4 = reinterpret_cast<const float4*>(sc + wk * kD + 16 * q);
+    if (16 * wk < nv) {
+      const float4* s4 = reinterpret_cast<const float4*>(sc + (wk >> 1) * kD + 16 * q);
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int ci = i ^ (swap ? 1 : 0);
@@ -225,8 +225,8 @@ __device__ __forceinline__ void decode_unit8(const unsigned char* u, unsigned ch
   }
   const u64 sub = pack2(-8388735.f, -8388735.f);
 #pragma unroll 2
-  for (int it = 0; it < 8; ++it) {
-    const int t = 32 * wk + 4 * it + tt;
+  for (int it = 0; it < 4; ++it) {
+    const int t = 16 * wk + 4 * it + tt;
     uint4 o[2];
     if (t < nv) {
       const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * kCb + 16 * q);
@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
       }
     } else if (warp >= 12) {
       // ======================= decode K/V to bf16 tiles =======================
-      const int wk = warp - 12;                          // 32-token group of each unit
+      const int wk = warp - 12;                          // 16-token slice of each unit
       Cursor kc, vc;
       kc.start(pre, p.B, H, cr);
       vc.start(pre, p.B, H, cr);
@@ -574,25 +574,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
           const u64 qs2 = pack2(p.qscale, p.qscale), nm2 = pack2(-m_ref, -m_ref);
           u64 z2 = 0ull;
 #pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t sr[64];
-            KVQ_LD32_AT(sr, 0, s_col + 64u * hh);
-            KVQ_LD32_AT(sr, 32, s_col + 64u * hh + 32u);
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t sr[32];
+            KVQ_LD32(sr, s_col + 32u * cc);
             tmem_wait_ld();
-            uint32_t pk[32];
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < 16; ++e) {
               const u64 x = fma2(pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), qs2, nm2);
               float p0 = ex2(lo_f(x)), p1 = ex2(hi_f(x));
               if (nv < kBT) {
-                p0 = 64 * hh + 2 * e < nv ? p0 : 0.f;
-                p1 = 64 * hh + 2 * e + 1 < nv ? p1 : 0.f;
+                p0 = 32 * cc + 2 * e < nv ? p0 : 0.f;
+                p1 = 32 * cc + 2 * e + 1 < nv ? p1 : 0.f;
               }
               z2 = add2(z2, pack2(p0, p1));
               pk[e] = pack_bf16(p0, p1);
             }
-            KVQ_ST16_AT(s_col + 32u * hh, pk, 0);
-            KVQ_ST16_AT(s_col + 32u * hh + 16u, pk, 16);
+            KVQ_ST16(s_col + 16u * cc, pk);
           }
           z += lo_f(z2) + hi_f(z2);
           tmem_wait_st();

@@ -26,7 +26,10 @@ struct MergeParams {
   unsigned int* err;
 };
 
-__global__ void __launch_bounds__(128) merge_kernel(MergeParams mp) {
+// Row-major merge: one CTA per (b, h), one thread per (row, feature), so
+// the parts' m and z (shared by a row's threads) and then their u values are
+// each fetched in one round of independent loads.
+__global__ void __launch_bounds__(512) merge_kernel(MergeParams mp) {
   extern __shared__ int s_pre[];                 // [B + 1]
   const MergeArgs& a = mp.a;
   if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
@@ -49,27 +52,29 @@ __global__ void __launch_bounds__(128) merge_kernel(MergeParams mp) {
   const long long E = S + nb;
   const long long c_first = S / cr.P, c_last = (E - 1) / cr.P;
   if (c_first == c_last) return;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int W = D + 2;
-  for (int r = warp; r < a.R; r += nwarps) {
+  const long long slot = static_cast<long long>(a.R_pad) * W;
+  for (int idx = threadIdx.x; idx < a.R * D; idx += blockDim.x) {
+    const int r = idx / D, d = idx % D;
+    const float* col = a.partials + (c_first + bh) * slot + static_cast<long long>(r) * W;   // part c: + (c - c_first) * slot
+    const int parts = static_cast<int>(c_last - c_first + 1);
     float m = -INFINITY;
-    for (long long c = c_first; c <= c_last; ++c) {
-      const float* part = a.partials + ((c + bh) * a.R_pad + r) * W;
-      if (part[1] > 0.f) m = fmaxf(m, part[0]);
+#pragma unroll 4
+    for (int c = 0; c < parts; ++c) {
+      const float zc = col[c * slot + 1], mc = col[c * slot];
+      if (zc > 0.f) m = fmaxf(m, mc);
     }
-    float z = 0.f;
-    for (long long c = c_first; c <= c_last; ++c) {
-      const float* part = a.partials + ((c + bh) * a.R_pad + r) * W;
-      if (part[1] > 0.f) z += expf(part[0] - m) * part[1];
-    }
-    for (int d = lane; d < D; d += 32) {
-      float u = 0.f;
-      for (long long c = c_first; c <= c_last; ++c) {
-        const float* part = a.partials + ((c + bh) * a.R_pad + r) * W;
-        if (part[1] > 0.f) u += expf(part[0] - m) * part[2 + d];
+    float z = 0.f, u = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < parts; ++c) {
+      const float zc = col[c * slot + 1], mc = col[c * slot], uc = col[c * slot + 2 + d];
+      if (zc > 0.f) {
+        const float w = expf(mc - m);
+        z = fmaf(w, zc, z);
+        u = fmaf(w, uc, u);
       }
-      store_from_f32(a.O, (row_base + r) * D + d, u / z, a.o_dtype);
     }
+    store_from_f32(a.O, (row_base + r) * D + d, u / z, a.o_dtype);
   }
 }
 
@@ -180,7 +185,9 @@ kvq_status launch_merge(const MergeArgs& a, cudaStream_t s) {
   if (blocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
   MergeParams mp{a, error_word()};
   if (!mp.err) return KVQ_ERR_CUDA;
-  merge_kernel<<<static_cast<unsigned>(blocks), 128, smem, s>>>(mp);
+  const long long work = static_cast<long long>(a.R) * a.D;
+  const int threads = work >= 512 ? 512 : static_cast<int>((work + 31) / 32 * 32);
+  merge_kernel<<<static_cast<unsigned>(blocks), threads, smem, s>>>(mp);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }

@@ -51,16 +51,52 @@ __global__ void __launch_bounds__(256) pack_k_kernel(PackParams p) {
   const long long head = static_cast<long long>(b) * p.H + h;
   const long long in_base = head * p.T * D;
   const int tt0 = gi * g;
-  for (int idx = threadIdx.x; idx < g * D; idx += blockDim.x) {
-    const int tt = tt0 + idx / D;
-    const int d = idx % D;
-    s_x[idx] = tt < p.T ? load_as_f32(p.X, in_base + static_cast<long long>(tt) * D + d, p.dtype) : 0.f;
+  // the group's g x D inputs into shared memory, loads issued in batches so
+  // their latencies overlap (float4 when the input is f32, 16-byte aligned
+  // and the group lies inside the range)
+  const int n = g * D;
+  const float* xf = static_cast<const float*>(p.X) + in_base + static_cast<long long>(tt0) * D;
+  if (p.dtype == KVQ_F32 && (D & 3) == 0 && tt0 + g <= p.T && (reinterpret_cast<uintptr_t>(xf) & 15u) == 0) {
+    const float4* src = reinterpret_cast<const float4*>(xf);
+    float4* dst = reinterpret_cast<float4*>(s_x);
+    constexpr int U = 4;
+    for (int i0 = 0; i0 < n / 4; i0 += U * static_cast<int>(blockDim.x)) {
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * static_cast<int>(blockDim.x) + threadIdx.x;
+        v[u] = i < n / 4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * static_cast<int>(blockDim.x) + threadIdx.x;
+        if (i < n / 4) dst[i] = v[u];
+      }
+    }
+  } else {
+    constexpr int U = 8;
+    for (int i0 = 0; i0 < n; i0 += U * static_cast<int>(blockDim.x)) {
+      float v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int idx = i0 + u * static_cast<int>(blockDim.x) + threadIdx.x;
+        const int tt = tt0 + idx / D;
+        v[u] = (idx < n && tt < p.T) ? load_as_f32(p.X, in_base + static_cast<long long>(tt) * D + idx % D, p.dtype)
+                                     : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int idx = i0 + u * static_cast<int>(blockDim.x) + threadIdx.x;
+        if (idx < n) s_x[idx] = v[u];
+      }
+    }
   }
   __syncthreads();
   float* s_scale = s_x + g * D;
   const long long kgroup = p.t0 / g + gi;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float amax = 0.f;
+#pragma unroll 8
     for (int tt = 0; tt < g; ++tt) amax = fmaxf(amax, fabsf(s_x[tt * D + d]));
     const float sc = group_scale(amax, qmax);
     s_scale[d] = sc;
