@@ -283,6 +283,7 @@ __device__ __forceinline__ float row_extreme(const uint32_t (&sr)[64]) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ CUtensorMap qmap, ChunkParams p) {
+  griddep_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_addr = su(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -732,9 +733,8 @@ kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   p.ctas = ctas;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
-  chunk_kernel<<<ctas, kThreads, smem, s>>>(qmap, p);
+  if (launch_pdl(chunk_kernel, dim3(ctas), dim3(kThreads), smem, s, qmap, p) != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
 
   MergeArgs m{};
   m.partials = p.partials;

@@ -292,6 +292,7 @@ __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem& ps,
 // the kernel
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
+  griddep_wait();
   extern __shared__ __align__(128) unsigned char smem_raw[];
   PairSmem* pairs = reinterpret_cast<PairSmem*>(smem_raw);
   float* qs = reinterpret_cast<float*>(pairs + kNP);    // [kG][kD], swizzled, * 1/eps
@@ -644,9 +645,9 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   p.ctas = ctas;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
-  decode_kernel<<<ctas, kThreads, smem, s>>>(p);
+  const cudaError_t le = launch_pdl(decode_kernel, dim3(ctas), dim3(kThreads), smem, s, p);
+  if (le != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
 
   MergeArgs m{};
   m.partials = p.partials;

@@ -48,6 +48,7 @@ size_t smem_bytes(int D, int B) {
 }
 
 __global__ void __launch_bounds__(kThreads) attend_generic_kernel(GenericParams p) {
+  griddep_wait();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int D = p.D;
   const int DS = D + 1;                               // padded row stride: no bank conflicts
@@ -244,9 +245,9 @@ kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
   p.O = a.O;
   p.partials = static_cast<float*>(a.workspace);
   p.ctas = ctas;
-  attend_generic_kernel<<<dim3(ctas, n_rt), kThreads, smem, s>>>(p);
+  const cudaError_t le = launch_pdl(attend_generic_kernel, dim3(ctas, n_rt), dim3(kThreads), smem, s, p);
+  if (le != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
-  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
 
   MergeArgs m{};
   m.partials = static_cast<const float*>(a.workspace);

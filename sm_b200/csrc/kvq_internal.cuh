@@ -1,5 +1,6 @@
 // Internal declarations shared by the CUDA sources of libkvq.so.
 #pragma once
+#include <utility>
 
 #include <cstddef>
 #include <cstdint>
@@ -37,6 +38,36 @@ struct Geometry {
 };
 
 bool make_geometry(const kvq_cache* c, Geometry* g);
+
+// ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+// Every kernel of the library is launched with launch_pdl, so its CTAs may
+// become resident while the previous kernel on the stream drains, and starts
+// with griddep_wait() -- which returns once every earlier grid on the stream
+// has completed and its memory is visible -- before any global-memory
+// access; it then lets the next kernel be scheduled.  Without a predecessor
+// (or without the launch attribute) both are no-ops.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------------------
 // dtype helpers

@@ -30,6 +30,7 @@ struct MergeParams {
 // the parts' m and z (shared by a row's threads) and then their u values are
 // each fetched in one round of independent loads.
 __global__ void __launch_bounds__(512) merge_kernel(MergeParams mp) {
+  griddep_wait();
   extern __shared__ int s_pre[];                 // [B + 1]
   const MergeArgs& a = mp.a;
   if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
@@ -88,6 +89,7 @@ constexpr int kFmBatch = 4;       // parts whose weights are held at once
 // 128-byte line; warp w owns 8 features.  The weights exp(m_c - m) of up to
 // four parts sit in registers and each part's 8 values are loaded together.
 __global__ void __launch_bounds__(kFmThreads, 4) merge_fm_kernel(MergeParams mp) {
+  griddep_wait();
   extern __shared__ int s_pre[];                   // [B + 1]
   const MergeArgs& a = mp.a;
   const int D = a.D;
@@ -175,10 +177,12 @@ kvq_status launch_merge(const MergeArgs& a, cudaStream_t s) {
       return KVQ_ERR_UNSUPPORTED;
     MergeParams mp{a, error_word()};
     if (!mp.err) return KVQ_ERR_CUDA;
-    merge_fm_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(chunks), static_cast<unsigned>(slices)),
-                      kFmThreads, smem, s>>>(mp);
+    if (launch_pdl(merge_fm_kernel,
+                   dim3(static_cast<unsigned>(bh), static_cast<unsigned>(chunks), static_cast<unsigned>(slices)),
+                   dim3(kFmThreads), smem, s, mp) != cudaSuccess)
+      return KVQ_ERR_CUDA;
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+    return KVQ_OK;
   }
   const size_t smem = static_cast<size_t>(a.B + 1) * sizeof(int);
   const long long blocks = static_cast<long long>(a.B) * a.H_kv;
@@ -187,9 +191,10 @@ kvq_status launch_merge(const MergeArgs& a, cudaStream_t s) {
   if (!mp.err) return KVQ_ERR_CUDA;
   const long long work = static_cast<long long>(a.R) * a.D;
   const int threads = work >= 512 ? 512 : static_cast<int>((work + 31) / 32 * 32);
-  merge_kernel<<<static_cast<unsigned>(blocks), threads, smem, s>>>(mp);
+  if (launch_pdl(merge_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), smem, s, mp) != cudaSuccess)
+    return KVQ_ERR_CUDA;
   count_launch();
-  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  return KVQ_OK;
 }
 
 }  // namespace kvq

@@ -44,6 +44,7 @@ struct PackParams {
 // each channel; the group's codes are g*D consecutive entries of the
 // flattened Np x D code matrix, so a 4-bit group owns whole bytes (g even).
 __global__ void __launch_bounds__(256) pack_k_kernel(PackParams p) {
+  griddep_wait();
   extern __shared__ float s_x[];                   // [g][D], then scale[D], 1/scale[D]
   const int gi = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = p.group, D = p.D;
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(256) pack_k_kernel(PackParams p) {
 // V: one thread per (token, group of g features).  Features beyond D are the
 // zero padding of the last group.
 __global__ void __launch_bounds__(256) pack_v_kernel(PackParams p) {
+  griddep_wait();
   const int ng = p.Dp / p.group;
   const long long total = static_cast<long long>(p.B) * p.H * p.T * ng;
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(256) pack_v_kernel(PackParams p) {
 // 4l..4l+3 (one 16-byte load), the 8 lanes of a group reduce the group max
 // with shuffles, and the lane writes its 4 codes (2 bytes, or 4 at 8 bits).
 __global__ void __launch_bounds__(256) pack_v128_kernel(PackParams p) {
+  griddep_wait();
   const long long rows = static_cast<long long>(p.B) * p.H * p.T;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -220,9 +223,8 @@ kvq_status launch_pack(const PackArgs& a, cudaStream_t s) {
                   static_cast<long long>(g.k_codes_head), static_cast<long long>(g.k_scales_head),
                   a.k_codes, a.k_scales};
     const dim3 kgrid((T + g.group - 1) / g.group, g.H_kv, g.B);
-    pack_k_kernel<<<kgrid, 256, smem, s>>>(pk);
+    if (launch_pdl(pack_k_kernel, kgrid, dim3(256), smem, s, pk) != cudaSuccess) return KVQ_ERR_CUDA;
     count_launch();
-    if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   }
   if (a.V) {
     PackParams pv{a.V, a.in_dtype, a.t0, T, g.bits, g.group, g.B, g.H_kv, g.D, g.Dp,
@@ -236,12 +238,14 @@ kvq_status launch_pack(const PackArgs& a, cudaStream_t s) {
       const long long rows = static_cast<long long>(g.B) * g.H_kv * T;
       const long long blocks = (rows + 7) / 8;
       if (blocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
-      pack_v128_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(pv);
+      if (launch_pdl(pack_v128_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, pv) != cudaSuccess)
+        return KVQ_ERR_CUDA;
     } else {
       const long long vthreads = static_cast<long long>(g.B) * g.H_kv * T * (g.Dp / g.group);
       const long long vblocks = (vthreads + 255) / 256;
       if (vblocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
-      pack_v_kernel<<<static_cast<unsigned>(vblocks), 256, 0, s>>>(pv);
+      if (launch_pdl(pack_v_kernel, dim3(static_cast<unsigned>(vblocks)), dim3(256), 0, s, pv) != cudaSuccess)
+        return KVQ_ERR_CUDA;
     }
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
