@@ -50,36 +50,50 @@ namespace {
 constexpr int kD = 128;
 constexpr int kG = 4;                 // query heads per KV head
 constexpr int kTB = 32;               // tokens per block (one K group)
-constexpr int kNP = 4;                // warp pairs per CTA
-constexpr int kS = 3;                 // pipeline stages per pair
-constexpr int kThreads = 2 * kNP * 32;
+// Per code width: warp pairs per CTA, pipeline stages per pair, code bytes
+// per token.  8-bit blocks carry twice the code bytes, so a CTA runs three
+// pairs of two stages to keep two CTAs on an SM.
+template <int BITS>
+struct Tr {
+  static constexpr int kNP = BITS == 4 ? 4 : 3;
+  static constexpr int kS = BITS == 4 ? 3 : 2;
+  static constexpr int kThreads = 2 * kNP * 32;
+  static constexpr int kCb = BITS == 4 ? 64 : 128;
+  // each channel's code f = 1 + code * eps sits in mantissa bits 15.. (even
+  // 4-bit channels, every 8-bit channel: eps = 2^-8) or 19.. (odd 4-bit
+  // channels: eps = 2^-4); corr = 1 + qmax * eps
+  static constexpr float kInvEpsEven = 256.f;
+  static constexpr float kInvEpsOdd = BITS == 4 ? 16.f : 256.f;
+  static constexpr float kCorrEven = BITS == 4 ? 1.f + 7.f / 256.f : 1.f + 127.f / 256.f;
+  static constexpr float kCorrOdd = BITS == 4 ? 1.f + 7.f / 16.f : 1.f + 127.f / 256.f;
+};
 constexpr int kPartStride = 36;       // floats per token row of score partials (8 x 4 + pad)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kCorrEven = 1.f + 7.f / 256.f;
-constexpr float kCorrOdd = 1.f + 7.f / 16.f;
 
+template <int BITS>
 struct Stage {
-  uint8_t kc[kTB * kD / 2];           // K codes, 64 B per token
-  uint8_t vc[kTB * kD / 2];           // V codes, 64 B per token
+  uint8_t kc[kTB * Tr<BITS>::kCb];    // K codes, 64 or 128 B per token
+  uint8_t vc[kTB * Tr<BITS>::kCb];    // V codes
   float ks[kD];                       // K scale row of the block's group
   float vs[kTB][kD / 32];             // V scales, 4 per token
 };
 
+template <int BITS>
 struct PairSmem {
-  Stage st[kS];
+  Stage<BITS> st[Tr<BITS>::kS];
   float part[2][kTB * kPartStride];   // score partials, double-buffered; part[0] holds the
                                       // V-warp's U at merge time
   float pv[kTB][20];                  // p' = p * s_v of token t, group g, head h at [t][4g + h];
                                       // four entries pad the row
-  unsigned long long full[kS];        // copies landed
-  unsigned long long empty[kS];       // V-warp done with the stage
+  unsigned long long full[Tr<BITS>::kS];    // copies landed
+  unsigned long long empty[Tr<BITS>::kS];   // V-warp done with the stage
   unsigned long long pfull[2];        // S-warp wrote part[i]
   unsigned long long pempty[2];       // V-warp read part[i]
 };
 
-static_assert(sizeof(Stage) % 16 == 0, "stage alignment");
-static_assert(sizeof(PairSmem) % 16 == 0, "pair alignment");
+static_assert(sizeof(Stage<4>) % 16 == 0 && sizeof(Stage<8>) % 16 == 0, "stage alignment");
+static_assert(sizeof(PairSmem<4>) % 16 == 0 && sizeof(PairSmem<8>) % 16 == 0, "pair alignment");
 static_assert(kTB * kPartStride >= kG * kD, "U must fit in a partials buffer");
 
 struct DecodeParams {
@@ -101,8 +115,10 @@ struct DecodeParams {
 
 // shared memory after the pairs: qs [kG][kD] (swizzled), mm/mz [kNP][kG],
 // mP [kNP][4 groups][kG], pre [B + 1], len [B]
+template <int BITS>
 size_t smem_bytes(int B) {
-  return sizeof(PairSmem) * kNP + sizeof(float) * (kG * kD + 2 * kNP * kG + kNP * 16) +
+  constexpr int kNP = Tr<BITS>::kNP;
+  return sizeof(PairSmem<BITS>) * kNP + sizeof(float) * (kG * kD + 2 * kNP * kG + kNP * 16) +
          sizeof(int) * (2 * B + 1);
 }
 
@@ -205,6 +221,40 @@ __device__ __forceinline__ void nibble_pairs(uint32_t w0, uint32_t w1, u64 f[8])
   }
 }
 
+// Channel pairs (16cs + 2i, 16cs + 2i + 1), i = 0..7, of a 16-byte load of
+// 8-bit codes: each byte shifted to mantissa bits 15..22 of 1.0, so
+// f = 1 + c * 2^-8 for every channel.
+__device__ __forceinline__ void byte_pairs15(const uint4& w4, u64 f[8]) {
+  const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t x = w[i >> 1];
+    const int r = 2 * (i & 1);
+    const uint32_t a = r == 0 ? (x << 15) : (x >> 1);            // byte r at bits 15..22
+    const uint32_t b = r == 0 ? (x << 7) : (x >> 9);             // byte r + 1
+    u64 v;
+    asm("{.reg .b32 t0, t1;\n\t"
+        "lop3.b32 t0, %1, 0x007F8000, 0x3F800000, 0xEA;\n\t"
+        "lop3.b32 t1, %2, 0x007F8000, 0x3F800000, 0xEA;\n\t"
+        "mov.b64 %0, {t0, t1};}"
+        : "=l"(v)
+        : "r"(a), "r"(b));
+    f[i] = v;
+  }
+}
+
+// The 16 channels (8 pairs) of lane slice cs of token t from a stage's codes.
+template <int BITS>
+__device__ __forceinline__ void code_pairs(const uint8_t* codes, int t, int cs, u64 f[8]) {
+  if (BITS == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(codes + t * 64 + cs * 8);
+    nibble_pairs(w.x, w.y, f);
+  } else {
+    const uint4 w = *reinterpret_cast<const uint4*>(codes + t * 128 + cs * 16);
+    byte_pairs15(w, f);
+  }
+}
+
 // q of the segment lives in shared memory pre-scaled by 1/eps, with the four
 // 16-byte chunks of each lane's 16 channels rotated so the eight lanes of a
 // quarter warp hit eight different bank groups.
@@ -269,19 +319,19 @@ __device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H
   return p;
 }
 
-__device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem& ps, int stage, int b,
+template <int BITS>
+__device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS>& ps, int stage, int b,
                                             int h, int j, const int* slen) {
   const long long head = static_cast<long long>(b) * p.H + h;
   const int len = slen[b];
   const int t0 = j * kTB;
   const int nv = min(kTB, len - t0);
-  Stage& st = ps.st[stage];
+  constexpr int kCb = Tr<BITS>::kCb;
+  Stage<BITS>& st = ps.st[stage];
   unsigned long long* bar = &ps.full[stage];
-  mbar_expect_tx(bar, 144u * nv + 512u);
-  bulk_g2s(st.kc, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * (kD / 2),
-           nv * (kD / 2), bar);
-  bulk_g2s(st.vc, p.v_codes + head * p.v_codes_head + static_cast<long long>(t0) * (kD / 2),
-           nv * (kD / 2), bar);
+  mbar_expect_tx(bar, static_cast<uint32_t>((2 * kCb + 16) * nv + 512));
+  bulk_g2s(st.kc, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
+  bulk_g2s(st.vc, p.v_codes + head * p.v_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
   bulk_g2s(st.ks, p.k_scales + head * p.k_scales_head + static_cast<long long>(j) * kD,
            kD * sizeof(float), bar);
   bulk_g2s(st.vs, p.v_scales + head * p.v_scales_head + static_cast<long long>(t0) * (kD / 32),
@@ -291,8 +341,12 @@ __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem& ps,
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
+template <int BITS>
+__global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodeParams p) {
   griddep_wait();
+  constexpr int kNP = Tr<BITS>::kNP, kS = Tr<BITS>::kS, kThreads = Tr<BITS>::kThreads;
+  using PairSmem = kvq::PairSmem<BITS>;
+  using Stage = kvq::Stage<BITS>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   PairSmem* pairs = reinterpret_cast<PairSmem*>(smem_raw);
   float* qs = reinterpret_cast<float*>(pairs + kNP);    // [kG][kD], swizzled, * 1/eps
@@ -334,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
   prod = prod_settle(prod, pre, p.B, H, cr, pair);
   if (is_s) {
     for (int s = 0; s < kS && prod.valid; ++s) {
-      if (lane == 0) issue_block(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
+      if (lane == 0) issue_block<BITS>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
       prod.j += kNP;
       prod = prod_settle(prod, pre, p.B, H, cr, pair);
     }
@@ -346,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
     const long long head = static_cast<long long>(b) * H + h;
     const long long qrow = static_cast<long long>(b) * H * kG + static_cast<long long>(h) * kG;
     for (int i = threadIdx.x; i < kG * kD; i += kThreads) {
-      const float ie = (i & 1) ? 16.f : 256.f;           // 1/eps of the channel's parity
+      const float ie = (i & 1) ? Tr<BITS>::kInvEpsOdd : Tr<BITS>::kInvEpsEven;   // 1/eps of the channel
       qs[qs_index(i / kD, i % kD)] = load_as_f32(p.Q, qrow * kD + i, p.q_dtype) * p.qscale * ie;
     }
     __syncthreads();
@@ -368,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
           ulonglong2 kv2[4];
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) kv2[jj] = ksv[jj];
-          const u64 corr = pack2(kCorrEven, kCorrOdd);
+          const u64 corr = pack2(Tr<BITS>::kCorrEven, Tr<BITS>::kCorrOdd);
 #pragma unroll
           for (int hh = 0; hh < kG; ++hh) {
             u64 c2 = 0ull;
@@ -390,9 +444,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
 #pragma unroll 2
         for (int it = 0; it < kTB / 4; ++it) {
           const int t = 4 * it + ts;
-          const uint2 kw = *reinterpret_cast<const uint2*>(st.kc + t * (kD / 2) + cs * 8);
           u64 f[8];
-          nibble_pairs(kw.x, kw.y, f);
+          code_pairs<BITS>(st.kc, t, cs, f);
           u64 acc[kG];
 #pragma unroll
           for (int hh = 0; hh < kG; ++hh) {
@@ -414,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
           wait_bar(&ps.empty[sp], (kp / kS) & 1u, p.err);
           if (lane == 0) {
             fence_proxy_async();
-            issue_block(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
+            issue_block<BITS>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
           }
           prod.j += kNP;
           prod = prod_settle(prod, pre, p.B, H, cr, pair);
@@ -498,9 +551,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
         for (int it = 0; it < kTB / 4; ++it) {
           const int t = 4 * it + ts;
           const float4 p4 = *reinterpret_cast<const float4*>(&ps.pv[t][4 * g]);
-          const uint2 vw = *reinterpret_cast<const uint2*>(st.vc + t * (kD / 2) + cs * 8);
           u64 f[8];
-          nibble_pairs(vw.x, vw.y, f);
+          code_pairs<BITS>(st.vc, t, cs, f);
           const u64 pp[kG] = {pack2(p4.x, p4.x), pack2(p4.y, p4.y), pack2(p4.z, p4.z),
                               pack2(p4.w, p4.w)};
           P[0] += p4.x;
@@ -565,8 +617,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
     const long long slot = static_cast<long long>(blockIdx.x) + head;
     for (int idx = threadIdx.x; idx < kG * kD; idx += kThreads) {
       const int hh = idx / kD, c = idx % kD;
-      const float corr = (c & 1) ? kCorrOdd : kCorrEven;
-      const float ie = (c & 1) ? 16.f : 256.f;
+      const float corr = (c & 1) ? Tr<BITS>::kCorrOdd : Tr<BITS>::kCorrEven;
+      const float ie = (c & 1) ? Tr<BITS>::kInvEpsOdd : Tr<BITS>::kInvEpsEven;
       float ms = -INFINITY;
 #pragma unroll
       for (int w = 0; w < kNP; ++w)
@@ -602,8 +654,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
 // host side
 // ---------------------------------------------------------------------------
 bool decode_applies(const AttendArgs& a) {
-  return a.g.bits == 4 && a.g.group == kTB && a.g.D == kD && a.Lq == 1 &&
-         a.H_q == kG * a.g.H_kv && smem_bytes(a.g.B) <= 113 * 1024;
+  return (a.g.bits == 4 || a.g.bits == 8) && a.g.group == kTB && a.g.D == kD && a.Lq == 1 &&
+         a.H_q == kG * a.g.H_kv &&
+         (a.g.bits == 4 ? smem_bytes<4>(a.g.B) : smem_bytes<8>(a.g.B)) <= 113 * 1024;
 }
 
 int decode_ctas(const AttendArgs& a) {
@@ -620,9 +673,12 @@ size_t decode_workspace(const AttendArgs& a) {
 
 kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   const int ctas = decode_ctas(a);
-  const size_t smem = smem_bytes(a.g.B);
-  if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  const bool b4 = a.g.bits == 4;
+  const size_t smem = b4 ? smem_bytes<4>(a.g.B) : smem_bytes<8>(a.g.B);
+  auto kernel = b4 ? decode_kernel<4> : decode_kernel<8>;
+  const int threads = b4 ? Tr<4>::kThreads : Tr<8>::kThreads;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
     return KVQ_ERR_CUDA;
   DecodeParams p{};
   p.Q = a.Q;
@@ -645,7 +701,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   p.ctas = ctas;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
-  const cudaError_t le = launch_pdl(decode_kernel, dim3(ctas), dim3(kThreads), smem, s, p);
+  const cudaError_t le = launch_pdl(kernel, dim3(ctas), dim3(threads), smem, s, p);
   if (le != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
 
@@ -667,7 +723,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   return launch_merge(m, s);
 }
 
-const AttendImpl kDecode{"decode_gqa4_d128_b4g32", decode_applies, decode_workspace, decode_launch};
+const AttendImpl kDecode{"decode_gqa4_d128_g32", decode_applies, decode_workspace, decode_launch};
 
 }  // namespace
 

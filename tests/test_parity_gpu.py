@@ -303,6 +303,16 @@ def test_decode_gqa_full(sm):
     _full_case(sm, "decode_gqa")
 
 
+def test_decode_gqa_full_8bit(sm):
+    """The decode workload with 8-bit codes (the tuned decode kernel's 8-bit
+    form), sampled heads against the oracle."""
+    q, k, v, lens, meta = W.gqa_case("decode_gqa", 0)
+    q = bf16_values(q)
+    small = pack_gpu(sm, np.ascontiguousarray(k[:1, :, :64]), np.ascontiguousarray(v[:1, :, :64]), 8, meta["group"])
+    assert sm.kernel_name(small, meta["H_q"], 1).startswith("decode_gqa4")
+    _check_gqa(sm, q, k, v, lens, 8, meta["group"], 1.0, heads=SAMPLE)
+
+
 def test_long_context_full(sm):
     _full_case(sm, "long_context", heads=[(0, 0), (3, 5), (7, 7), (6, 2)])
 
