@@ -478,7 +478,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD,
                     help="the decode GQA workload is the headline; the others are for study")
     ap.add_argument("--bits", type=int, choices=[4, 8], default=0,
-                    help="code width for the chunk workload (default 4)")
+                    help="code width (default: the workload's, 4 for the chunk workload)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
