@@ -38,8 +38,9 @@
 // f = 1 + n * eps with eps = 2^-8 for even channels and 2^-4 for odd ones,
 // and the two channels of a byte land in one f32x2 pair.  With q'' = q' / eps,
 // sum q'' f - sum q'' (1 + 7 eps) = sum q' (n - 7): the second sum is one
-// correction per block.  For V, u = (U - (1 + 7 eps) P) / eps with U = sum p' f
-// and P = sum p'.  Rounding error is amplified by at most 2^8 / 7.
+// correction per block.  For V the subtraction is done per channel pair,
+// f - (1 + 7 eps) = (n - 7) eps, which is exact, so u = sum p' (n - 7) eps
+// carries no cancellation and a zero code contributes exactly zero.
 #include "f32x2.cuh"
 #include "kvq_internal.cuh"
 #include "plan.cuh"
@@ -114,11 +115,11 @@ struct DecodeParams {
 };
 
 // shared memory after the pairs: qs [kG][kD] (swizzled), mm/mz [kNP][kG],
-// mP [kNP][4 groups][kG], pre [B + 1], len [B]
+// pre [B + 1], len [B]
 template <int BITS>
 size_t smem_bytes(int B) {
   constexpr int kNP = Tr<BITS>::kNP;
-  return sizeof(PairSmem<BITS>) * kNP + sizeof(float) * (kG * kD + 2 * kNP * kG + kNP * 16) +
+  return sizeof(PairSmem<BITS>) * kNP + sizeof(float) * (kG * kD + 2 * kNP * kG) +
          sizeof(int) * (2 * B + 1);
 }
 
@@ -352,8 +353,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
   float* qs = reinterpret_cast<float*>(pairs + kNP);    // [kG][kD], swizzled, * 1/eps
   float* mm = qs + kG * kD;                              // [kNP][kG] pair maxima
   float* mz = mm + kNP * kG;                             // [kNP][kG] pair sums
-  float* mP = mz + kNP * kG;                             // [kNP][4][kG] pair sums of p'
-  int* pre = reinterpret_cast<int*>(mP + kNP * 16);      // [B + 1]
+  int* pre = reinterpret_cast<int*>(mz + kNP * kG);     // [B + 1]
   int* slen = pre + p.B + 1;                             // [B] lengths clamped to [0, N_cap]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -476,16 +476,16 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
     } else {
       // ===================== V-warp: softmax and values =====================
       u64 u[kG][8];
-      float m[kG], z[kG], P[kG];                        // z: per token-lane; P: per (ts, cs) lane
+      float m[kG], z[kG];                               // z: per token-lane
 #pragma unroll
       for (int hh = 0; hh < kG; ++hh) {
         m[hh] = -INFINITY;
         z[hh] = 0.f;
-        P[hh] = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) u[hh][i] = 0ull;
       }
       const int g = cs >> 1;                            // V group of channels 16cs..16cs+15
+      const u64 ncorr = pack2(-Tr<BITS>::kCorrEven, -Tr<BITS>::kCorrOdd);
       for (int j = seg.jb + pair; j < seg.je; j += kNP, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
@@ -525,7 +525,6 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
         if (grow) {                                     // warp-uniform
 #pragma unroll
           for (int hh = 0; hh < kG; ++hh) {
-            P[hh] *= a[hh];
             const u64 a2 = pack2(a[hh], a[hh]);
 #pragma unroll
             for (int i = 0; i < 8; ++i) u[hh][i] = mul2(u[hh][i], a2);
@@ -555,10 +554,10 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
           code_pairs<BITS>(st.vc, t, cs, f);
           const u64 pp[kG] = {pack2(p4.x, p4.x), pack2(p4.y, p4.y), pack2(p4.z, p4.z),
                               pack2(p4.w, p4.w)};
-          P[0] += p4.x;
-          P[1] += p4.y;
-          P[2] += p4.z;
-          P[3] += p4.w;
+          // f - (1 + qmax eps) = (code - qmax) eps exactly, so a zero code
+          // contributes exactly zero
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] = add2(f[i], ncorr);
 #pragma unroll
           for (int hh = 0; hh < kG; ++hh)
 #pragma unroll
@@ -568,13 +567,11 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
         if (lane == 0) mbar_arrive(&ps.empty[stage]);
       }
 
-      // pair state: z per token-lane; U and P per (ts, cs) lane -> reduce over ts
+      // pair state: z per token-lane; u per (ts, cs) lane -> reduce over ts
 #pragma unroll
       for (int hh = 0; hh < kG; ++hh) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) z[hh] += __shfl_xor_sync(0xffffffffu, z[hh], o);
-        P[hh] += __shfl_xor_sync(0xffffffffu, P[hh], 8);
-        P[hh] += __shfl_xor_sync(0xffffffffu, P[hh], 16);
       }
       if (lane == 0) {
 #pragma unroll
@@ -582,10 +579,6 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
           mm[pair * kG + hh] = m[hh];
           mz[pair * kG + hh] = z[hh];
         }
-      }
-      if (ts == 0 && (cs & 1) == 0) {
-#pragma unroll
-        for (int hh = 0; hh < kG; ++hh) mP[(pair * 4 + g) * kG + hh] = P[hh];
       }
       float uf[kG][16];
 #pragma unroll
@@ -617,7 +610,6 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
     const long long slot = static_cast<long long>(blockIdx.x) + head;
     for (int idx = threadIdx.x; idx < kG * kD; idx += kThreads) {
       const int hh = idx / kD, c = idx % kD;
-      const float corr = (c & 1) ? Tr<BITS>::kCorrOdd : Tr<BITS>::kCorrEven;
       const float ie = (c & 1) ? Tr<BITS>::kInvEpsOdd : Tr<BITS>::kInvEpsEven;
       float ms = -INFINITY;
 #pragma unroll
@@ -629,7 +621,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
         const float zw = mz[w * kG + hh];
         if (zw > 0.f) {
           const float f = ex2(mm[w * kG + hh] - ms);
-          const float uw = (pairs[w].part[0][hh * kD + c] - corr * mP[(w * 4 + c / 32) * kG + hh]) * ie;
+          const float uw = pairs[w].part[0][hh * kD + c] * ie;
           zt += f * zw;
           ut += f * uw;
         }

@@ -250,6 +250,21 @@ def test_decode_bad_lengths(sm):
     sm.check()
 
 
+@pytest.mark.parametrize("hq,lq,bits", [(8, 1, 4), (8, 1, 8), (8, 32, 4), (8, 32, 8), (2, 1, 4)])
+@pytest.mark.parametrize("zero_k", [True, False])
+def test_zero_values_give_exact_zero(sm, hq, lq, bits, zero_k):
+    """A zero V cache (every group's scale 1, every code qmax) decodes to
+    exact zeros, so every output row is exactly zero: the tolerance
+    2e-3 * max|V| is 0 here.  With K zero too every score is 0; with K random
+    the softmax is not uniform.  Decode (4/8-bit), chunk and generic kernels."""
+    q, k, v, lens = _gqa_case(2, hq, 2, 300, 128, [300, 157], lq=lq, seed=50 + bits, bits=bits)
+    v[:] = 0.0
+    if zero_k:
+        k[:] = 0.0
+    o = _check_gqa(sm, q, k, v, lens, bits, 32, 1.0)
+    assert np.all(o == 0.0)
+
+
 def test_repeat_is_bit_identical(sm):
     q, k, v, lens = _gqa_case(2, 8, 2, 300, 128, [300, 200], seed=6)
     cache = pack_gpu(sm, k, v, 4, 32)
