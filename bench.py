@@ -123,17 +123,21 @@ def measured_peaks(kind: str = "hbm"):
 
 
 PROFILE_FOR = {
-    "decode_gqa": "attend_decode_gqa_b32_ctx4096.md",
-    "long_context": "attend_decode_long_context_b8.md",
-    "chunk": "attend_chunk_b4_lq64_ctx16384.md",
+    ("decode_gqa", 4): "attend_decode_gqa_b32_ctx4096.md",
+    ("decode_gqa", 8): "attend_decode_gqa_b32_ctx4096_8bit.md",
+    ("chunk", 4): "attend_chunk_b4_lq64_ctx16384.md",
 }
 
 
-def recorded_traffic(kernel_src: str, workload: str = "decode_gqa"):
+def recorded_traffic(kernel_src: str, workload: str = "decode_gqa", bits: int = 4):
     """Per-launch DRAM bytes of the attend kernel from the committed ncu
-    summary, or None when the kernel source changed since the capture."""
+    summary of this workload and code width, or None when there is none or
+    the kernel source changed since the capture."""
     import hashlib
-    summary = os.path.join(ROOT, "profiles", PROFILE_FOR.get(workload, ""))
+    name = PROFILE_FOR.get((workload, bits))
+    if name is None:
+        return None
+    summary = os.path.join(ROOT, "profiles", name)
     try:
         text = open(summary, encoding="utf-8").read()
         src = open(kernel_src, "rb").read()
@@ -456,7 +460,7 @@ def run_kvq(args, rank, world, local_rank):
                          "algorithmic_bytes_per_launch": abytes,
                          "algorithmic_flops_per_launch": attend_flops,
                          "attend_gbs": round(abytes / (att_ms * 1e-3) / 1e9, 1),
-                         "traffic": recorded_traffic(src, workload)},
+                         "traffic": recorded_traffic(src, workload, bits)},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_max / args.steps * 1e3, 3)},
             "gpu_launches": int(launches),
