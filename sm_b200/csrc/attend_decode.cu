@@ -57,6 +57,7 @@ constexpr int kTB = 32;               // tokens per block (one K group)
 template <int BITS>
 struct Tr {
   static constexpr int kNP = BITS == 4 ? 4 : 3;
+  static constexpr int kCtasPerSm = 2;
   static constexpr int kS = BITS == 4 ? 3 : 2;
   static constexpr int kThreads = 2 * kNP * 32;
   static constexpr int kCb = BITS == 4 ? 64 : 128;
@@ -68,7 +69,6 @@ struct Tr {
   static constexpr float kCorrEven = BITS == 4 ? 1.f + 7.f / 256.f : 1.f + 127.f / 256.f;
   static constexpr float kCorrOdd = BITS == 4 ? 1.f + 7.f / 16.f : 1.f + 127.f / 256.f;
 };
-constexpr int kPartStride = 36;       // floats per token row of score partials (8 x 4 + pad)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -83,8 +83,9 @@ struct Stage {
 template <int BITS>
 struct PairSmem {
   Stage<BITS> st[Tr<BITS>::kS];
-  float part[2][kTB * kPartStride];   // score partials, double-buffered; part[0] holds the
-                                      // V-warp's U at merge time
+  float qs[kG * kD];                  // q of the pair's current segment, * scale * log2e / eps,
+                                      // swizzled (qs_index)
+  float part[2][kTB * 32];            // score partials, double-buffered (part_index)
   float pv[kTB][20];                  // p' = p * s_v of token t, group g, head h at [t][4g + h];
                                       // four entries pad the row
   unsigned long long full[Tr<BITS>::kS];    // copies landed
@@ -95,7 +96,6 @@ struct PairSmem {
 
 static_assert(sizeof(Stage<4>) % 16 == 0 && sizeof(Stage<8>) % 16 == 0, "stage alignment");
 static_assert(sizeof(PairSmem<4>) % 16 == 0 && sizeof(PairSmem<8>) % 16 == 0, "pair alignment");
-static_assert(kTB * kPartStride >= kG * kD, "U must fit in a partials buffer");
 
 struct DecodeParams {
   const void* Q;
@@ -110,17 +110,14 @@ struct DecodeParams {
   float qscale;                       // scale * log2(e)
   void* O;
   float* partials;                    // [slots][kG][kD + 2]
-  int ctas;
+  int ctas;                           // CTAs; each warp pair is one worker of the plan
   unsigned int* err;
 };
 
-// shared memory after the pairs: qs [kG][kD] (swizzled), mm/mz [kNP][kG],
-// pre [B + 1], len [B]
+// shared memory after the pairs: pre [B + 1], len [B]
 template <int BITS>
 size_t smem_bytes(int B) {
-  constexpr int kNP = Tr<BITS>::kNP;
-  return sizeof(PairSmem<BITS>) * kNP + sizeof(float) * (kG * kD + 2 * kNP * kG) +
-         sizeof(int) * (2 * B + 1);
+  return sizeof(PairSmem<BITS>) * Tr<BITS>::kNP + sizeof(int) * (2 * B + 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -173,10 +170,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -264,8 +257,13 @@ __device__ __forceinline__ int qs_index(int h, int c) {
   return h * kD + cs * 16 + ((j ^ ((cs >> 1) & 3)) << 2) + (c & 3);
 }
 
+// Score partials of token t: the eight channel slices' float4 (one value per
+// head) in a 128-byte row, slice i at float4 (i ^ (t & 7)) so that eight
+// lanes reading slice i of eight tokens hit eight different bank groups.
+__device__ __forceinline__ int part_index(int t, int i) { return t * 32 + ((i ^ (t & 7)) << 2); }
+
 // ---------------------------------------------------------------------------
-// iteration over the CTA's block range
+// iteration over a worker's block range
 // ---------------------------------------------------------------------------
 struct Seg {
   int b, h, nb, jb, je;
@@ -310,16 +308,17 @@ struct Prod {
   bool valid;
 };
 
-__device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H, const CtaRange& cr,
-                                            int pair) {
+__device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H, const CtaRange& cr) {
   while (p.valid && p.j >= p.seg.je) {
     p.seg = next_seg(p.seg, pre, B, H, cr);
     p.valid = p.seg.valid;
-    p.j = p.seg.jb + pair;
+    p.j = p.seg.jb;
   }
   return p;
 }
 
+// Lane 0 arms the stage's barrier with the block's byte count and issues the
+// four copies: K codes, V codes, the K scale row and the V scales.
 template <int BITS>
 __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS>& ps, int stage, int b,
                                             int h, int j, const int* slen) {
@@ -343,17 +342,14 @@ __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS
 // the kernel
 // ---------------------------------------------------------------------------
 template <int BITS>
-__global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) decode_kernel(DecodeParams p) {
   griddep_wait();
   constexpr int kNP = Tr<BITS>::kNP, kS = Tr<BITS>::kS, kThreads = Tr<BITS>::kThreads;
   using PairSmem = kvq::PairSmem<BITS>;
   using Stage = kvq::Stage<BITS>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   PairSmem* pairs = reinterpret_cast<PairSmem*>(smem_raw);
-  float* qs = reinterpret_cast<float*>(pairs + kNP);    // [kG][kD], swizzled, * 1/eps
-  float* mm = qs + kG * kD;                              // [kNP][kG] pair maxima
-  float* mz = mm + kNP * kG;                             // [kNP][kG] pair sums
-  int* pre = reinterpret_cast<int*>(mz + kNP * kG);     // [B + 1]
+  int* pre = reinterpret_cast<int*>(pairs + kNP);       // [B + 1]
   int* slen = pre + p.B + 1;                             // [B] lengths clamped to [0, N_cap]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -379,36 +375,65 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
 
+  // From here on every warp pair works alone: it is worker blockIdx.x * kNP +
+  // pair of the plan, with a contiguous block range of its own, and no
+  // CTA-wide barrier follows.
   const int H = p.H;
-  const CtaRange cr = cta_range(pre, p.B, H, p.ctas, blockIdx.x);
+  const int worker = blockIdx.x * kNP + pair;
+  const CtaRange cr = cta_range(pre, p.B, H, p.ctas * kNP, worker);
   if (cr.g0 >= cr.g1) return;
 
   Seg seg = first_seg(pre, p.B, H, cr);
-  Prod prod{seg, seg.jb + pair, true};
-  prod = prod_settle(prod, pre, p.B, H, cr, pair);
+  Prod prod{seg, seg.jb, true};
+  prod = prod_settle(prod, pre, p.B, H, cr);
+  // S-warp: q of a segment, loaded (lane + 32 r) before it is scaled into qs.
+  // The first segment's loads go out before the first block copies so they
+  // do not queue behind them.
+  constexpr int kPer = kG * kD / 32;
+  float qv[kPer];
+  auto load_q = [&](const Seg& sg) {
+    const long long qrow = (static_cast<long long>(sg.b) * H + sg.h) * kG;
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) qv[r] = load_as_f32(p.Q, qrow * kD + lane + 32 * r, p.q_dtype);
+  };
+  // q * scale * log2e / eps into the pair's qs (the channel of value r is
+  // lane + 32 r, so its parity is the lane's)
+  auto store_q = [&]() {
+    const float qf = p.qscale * ((lane & 1) ? Tr<BITS>::kInvEpsOdd : Tr<BITS>::kInvEpsEven);
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int i = lane + 32 * r;
+      ps.qs[qs_index(i / kD, i % kD)] = qv[r] * qf;
+    }
+  };
   if (is_s) {
+    load_q(seg);
     for (int s = 0; s < kS && prod.valid; ++s) {
       if (lane == 0) issue_block<BITS>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
-      prod.j += kNP;
-      prod = prod_settle(prod, pre, p.B, H, cr, pair);
+      ++prod.j;
+      prod = prod_settle(prod, pre, p.B, H, cr);
     }
+    store_q();
   }
 
   uint32_t k = 0;                                        // blocks this pair has consumed
+  bool first = true;
   while (seg.valid) {
     const int b = seg.b, h = seg.h;
     const long long head = static_cast<long long>(b) * H + h;
     const long long qrow = static_cast<long long>(b) * H * kG + static_cast<long long>(h) * kG;
-    for (int i = threadIdx.x; i < kG * kD; i += kThreads) {
-      const float ie = (i & 1) ? Tr<BITS>::kInvEpsOdd : Tr<BITS>::kInvEpsEven;   // 1/eps of the channel
-      qs[qs_index(i / kD, i % kD)] = load_as_f32(p.Q, qrow * kD + i, p.q_dtype) * p.qscale * ie;
-    }
-    __syncthreads();
     const int len = slen[b];
 
     if (is_s) {
       // ===================== S-warp: partial scores =====================
-      for (int j = seg.jb + pair; j < seg.je; j += kNP, ++k) {
+      // the segment's q, pre-scaled by 1/eps; only this warp reads it
+      float* qs = ps.qs;
+      if (!first) {
+        load_q(seg);
+        store_q();
+      }
+      __syncwarp();
+      for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
         wait_bar(&ps.full[stage], (k / kS) & 1u, p.err);
@@ -453,7 +478,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
 #pragma unroll
             for (int i = 1; i < 8; ++i) acc[hh] = fma2(q2[hh][i], f[i], acc[hh]);
           }
-          *reinterpret_cast<float4*>(part + t * kPartStride + cs * 4) =
+          *reinterpret_cast<float4*>(part + part_index(t, cs)) =
               make_float4(lo_f(acc[0]) + hi_f(acc[0]), lo_f(acc[1]) + hi_f(acc[1]),
                           lo_f(acc[2]) + hi_f(acc[2]), lo_f(acc[3]) + hi_f(acc[3]));
         }
@@ -464,13 +489,12 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
         if (k > 0 && prod.valid) {
           const uint32_t kp = k - 1;
           const int sp = static_cast<int>(kp % kS);
+          // the V-warp's reads of the stage happen before its arrive on
+          // `empty`, which this wait acquires: the copy cannot overtake them
           wait_bar(&ps.empty[sp], (kp / kS) & 1u, p.err);
-          if (lane == 0) {
-            fence_proxy_async();
-            issue_block<BITS>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
-          }
-          prod.j += kNP;
-          prod = prod_settle(prod, pre, p.B, H, cr, pair);
+          if (lane == 0) issue_block<BITS>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
+          ++prod.j;
+          prod = prod_settle(prod, pre, p.B, H, cr);
         }
       }
     } else {
@@ -486,7 +510,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
       }
       const int g = cs >> 1;                            // V group of channels 16cs..16cs+15
       const u64 ncorr = pack2(-Tr<BITS>::kCorrEven, -Tr<BITS>::kCorrOdd);
-      for (int j = seg.jb + pair; j < seg.je; j += kNP, ++k) {
+      for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
         wait_bar(&ps.full[stage], (k / kS) & 1u, p.err);
@@ -499,7 +523,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
         const float* part = ps.part[pb];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float4 v = *reinterpret_cast<const float4*>(part + lane * kPartStride + 4 * i);
+          const float4 v = *reinterpret_cast<const float4*>(part + part_index(lane, i));
           s[0] += v.x;
           s[1] += v.y;
           s[2] += v.z;
@@ -567,77 +591,50 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
         if (lane == 0) mbar_arrive(&ps.empty[stage]);
       }
 
-      // pair state: z per token-lane; u per (ts, cs) lane -> reduce over ts
+      // the pair's state for the segment: z summed over the token lanes, u
+      // over the four token groups; lanes with ts = 0 hold channels 16cs..
 #pragma unroll
       for (int hh = 0; hh < kG; ++hh) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) z[hh] += __shfl_xor_sync(0xffffffffu, z[hh], o);
       }
-      if (lane == 0) {
+      const bool whole = (seg.jb == 0) && (seg.je == seg.nb);
+      const long long slot = static_cast<long long>(worker) + head;
 #pragma unroll
-        for (int hh = 0; hh < kG; ++hh) {
-          mm[pair * kG + hh] = m[hh];
-          mz[pair * kG + hh] = z[hh];
-        }
-      }
-      float uf[kG][16];
-#pragma unroll
-      for (int hh = 0; hh < kG; ++hh)
+      for (int hh = 0; hh < kG; ++hh) {
+        float uf[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          float x = lo_f(u[hh][i]), y = hi_f(u[hh][i]);
+          // u carries a factor eps of the channel: scale it back
+          float x = lo_f(u[hh][i]) * Tr<BITS>::kInvEpsEven, y = hi_f(u[hh][i]) * Tr<BITS>::kInvEpsOdd;
           x += __shfl_xor_sync(0xffffffffu, x, 8);
           y += __shfl_xor_sync(0xffffffffu, y, 8);
           x += __shfl_xor_sync(0xffffffffu, x, 16);
           y += __shfl_xor_sync(0xffffffffu, y, 16);
-          uf[hh][2 * i] = x;
-          uf[hh][2 * i + 1] = y;
+          uf[2 * i] = x;
+          uf[2 * i + 1] = y;
         }
-      if (ts == 0) {
+        if (ts != 0) continue;
+        if (whole) {
+          // the worker covered the whole (b, h): O = u / z
+          const float iz = 1.f / z[hh];
 #pragma unroll
-        for (int hh = 0; hh < kG; ++hh) {
-          float4* dst = reinterpret_cast<float4*>(ps.part[0] + hh * kD + 16 * cs);
+          for (int c = 0; c < 16; ++c)
+            store_from_f32(p.O, (qrow + hh) * kD + 16 * cs + c, uf[c] * iz, p.q_dtype);
+        } else {
+          float* part = p.partials + (slot * kG + hh) * (kD + 2);
+          if (cs == 0) {
+            part[0] = m[hh] * kLn2;
+            part[1] = z[hh];
+          }
+          // 8-byte stores: the row of kD + 2 floats keeps only 8-byte alignment
+          float2* dst = reinterpret_cast<float2*>(part + 2 + 16 * cs);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_float4(uf[hh][4 * q], uf[hh][4 * q + 1], uf[hh][4 * q + 2], uf[hh][4 * q + 3]);
+          for (int q = 0; q < 8; ++q) dst[q] = make_float2(uf[2 * q], uf[2 * q + 1]);
         }
       }
     }
-    __syncthreads();
-
-    // ---- merge the pairs: thread -> (head, channel)
-    const bool whole = (seg.jb == 0) && (seg.je == seg.nb);
-    const long long slot = static_cast<long long>(blockIdx.x) + head;
-    for (int idx = threadIdx.x; idx < kG * kD; idx += kThreads) {
-      const int hh = idx / kD, c = idx % kD;
-      const float ie = (c & 1) ? Tr<BITS>::kInvEpsOdd : Tr<BITS>::kInvEpsEven;
-      float ms = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kNP; ++w)
-        if (mz[w * kG + hh] > 0.f) ms = fmaxf(ms, mm[w * kG + hh]);
-      float zt = 0.f, ut = 0.f;
-#pragma unroll
-      for (int w = 0; w < kNP; ++w) {
-        const float zw = mz[w * kG + hh];
-        if (zw > 0.f) {
-          const float f = ex2(mm[w * kG + hh] - ms);
-          const float uw = pairs[w].part[0][hh * kD + c] * ie;
-          zt += f * zw;
-          ut += f * uw;
-        }
-      }
-      if (whole) {
-        store_from_f32(p.O, (qrow + hh) * kD + c, ut / zt, p.q_dtype);
-      } else {
-        float* part = p.partials + (slot * kG + hh) * (kD + 2);
-        if (c == 0) {
-          part[0] = ms * kLn2;
-          part[1] = zt;
-        }
-        part[2 + c] = ut;
-      }
-    }
-    __syncthreads();
+    first = false;
     seg = next_seg(seg, pre, p.B, H, cr);
   }
 }
@@ -645,22 +642,30 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, 2) decode_kernel(DecodePar
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+// Shared memory one CTA may use so that Tr::kCtasPerSm of them fit an SM
+// (228 KB per SM, 1 KB of it reserved per CTA, at most 227 KB per CTA).
+constexpr size_t kSmemPerCta = 113 * 1024;
+
 bool decode_applies(const AttendArgs& a) {
   return (a.g.bits == 4 || a.g.bits == 8) && a.g.group == kTB && a.g.D == kD && a.Lq == 1 &&
          a.H_q == kG * a.g.H_kv &&
-         (a.g.bits == 4 ? smem_bytes<4>(a.g.B) : smem_bytes<8>(a.g.B)) <= 113 * 1024;
+         (a.g.bits == 4 ? smem_bytes<4>(a.g.B) : smem_bytes<8>(a.g.B)) <= kSmemPerCta;
 }
 
 int decode_ctas(const AttendArgs& a) {
   const long long t_max = static_cast<long long>(a.g.B) * a.g.H_kv * ((a.g.N_cap + kTB - 1) / kTB);
-  long long ctas = a.splits > 0 ? a.splits : 2LL * (sm_count() > 0 ? sm_count() : 148);
+  const int per_sm = a.g.bits == 4 ? Tr<4>::kCtasPerSm : Tr<8>::kCtasPerSm;
+  long long ctas = a.splits > 0 ? a.splits : static_cast<long long>(per_sm) * (sm_count() > 0 ? sm_count() : 148);
   if (ctas > t_max) ctas = t_max;
   if (ctas < 1) ctas = 1;
   return static_cast<int>(ctas);
 }
 
+// Warp pairs per CTA: each pair is one worker of the plan.
+int decode_pairs(const AttendArgs& a) { return a.g.bits == 4 ? Tr<4>::kNP : Tr<8>::kNP; }
+
 size_t decode_workspace(const AttendArgs& a) {
-  return partial_slots(decode_ctas(a), a.g.B, a.g.H_kv) * kG * (kD + 2) * sizeof(float);
+  return partial_slots(decode_ctas(a) * decode_pairs(a), a.g.B, a.g.H_kv) * kG * (kD + 2) * sizeof(float);
 }
 
 kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
@@ -706,7 +711,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   m.H_kv = a.g.H_kv;
   m.N_cap = a.g.N_cap;
   m.BT = kTB;
-  m.ctas = ctas;
+  m.ctas = ctas * decode_pairs(a);
   m.R = kG;
   m.R_pad = kG;
   m.D = kD;
