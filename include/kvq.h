@@ -134,14 +134,47 @@ KVQ_API kvq_status kvq_pack(const void* K, const void* V, kvq_dtype in_dtype, in
  *   splits   how many CTAs share the concatenated (b, h, token-block) list;
  *            0 = automatic (a multiple of the SM count).  Any value gives the
  *            same result up to float rounding order.
- * A length outside 1..N_cap is recorded for kvq_check (KVQ_ERR_LENGTH); the
- * rows of that sequence are then written as zeros.
+ * A length outside 1..N_cap is recorded for kvq_check (KVQ_ERR_LENGTH): a
+ * length below 1 gives zero rows, one above N_cap is read as N_cap.
  * Errors: KVQ_ERR_ARG, KVQ_ERR_ALIGN, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA,
  * KVQ_ERR_UNSUPPORTED (D > 256).
  */
 KVQ_API kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
                       const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
                       void* workspace, size_t ws_bytes, int32_t splits, void* stream);
+
+/*
+ * Attention of Q over the packed cache followed by a window of recent tokens
+ * kept unquantized.  The pages leave this as their next study: keep the same
+ * packed format and spend a limited high-precision budget on the most recent
+ * tokens ("KV分组打包：4-bit到底省了多少？", section "小练习与常见错误", last
+ * paragraph).  The keys of sequence b are its packed tokens [0, lengths[b])
+ * followed by its window tokens [0, win_lengths[b]); each query row takes one
+ * softmax over all of them.
+ *   Q, cache, H_q, Lq, scale, O, workspace, ws_bytes, splits: as kvq_attend,
+ *            except that the workspace must hold kvq_workspace_size_window(...)
+ *            bytes.
+ *   lengths      device int32 [B]: packed keys of each sequence, 0..N_cap.
+ *   K_win, V_win device, [B, H_kv, W_cap, D] in win_dtype (KVQ_F32 or
+ *                KVQ_BF16), element (b, h, t, d) at ((b*H_kv + h)*W_cap + t)*D
+ *                + d; caller-owned, read only.
+ *   win_lengths  device int32 [B]: window keys of each sequence, 0..W_cap.
+ *   W_cap        window capacity per sequence, >= 1.
+ * A sequence with lengths outside 0..N_cap, win_lengths outside 0..W_cap, or
+ * no key at all is recorded for kvq_check (KVQ_ERR_LENGTH); lengths are read
+ * clamped to their ranges, and a sequence with no key gets zero rows.  The
+ * call launches the packed-cache kernel, a small kernel for the window's
+ * share and the split merge, which every sequence goes through.
+ * Errors: as kvq_attend.
+ */
+KVQ_API kvq_status kvq_attend_window(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                     const int32_t* lengths, const void* K_win, const void* V_win,
+                                     kvq_dtype win_dtype, const int32_t* win_lengths, int32_t W_cap,
+                                     int32_t H_q, int32_t Lq, float scale, void* O, void* workspace,
+                                     size_t ws_bytes, int32_t splits, void* stream);
+
+/* Workspace bytes kvq_attend_window needs (host); 0 for invalid arguments. */
+KVQ_API size_t kvq_workspace_size_window(const kvq_cache* cache, int32_t H_q, int32_t Lq, int32_t splits);
 
 /*
  * kvq_attend without a caller workspace, for callers that cannot allocate

@@ -49,6 +49,7 @@ from .kvq_oracle import (  # noqa: F401
     partial_state,
     attend_gqa,
     attend_gqa_heads,
+    attend_gqa_window,
     rel_l2_error,
     pack_cache,
 )

@@ -424,6 +424,43 @@ def attend_gqa(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray,
     return out
 
 
+def attend_gqa_window(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, lengths,
+                      k_win: np.ndarray, v_win: np.ndarray, win_lengths, scale: float) -> np.ndarray:
+    """Grouped-query attention over a packed cache plus a window of recent
+    tokens kept unquantized.
+
+    The pages leave this as the next study: keep the same packed format and
+    spend a limited high-precision budget on the most recent tokens
+    ("KV分组打包：4-bit到底省了多少？", section "小练习与常见错误", last
+    paragraph).  Reading taken here: the keys of sequence b are its decoded
+    packed tokens [0, lengths[b]) followed by its window tokens
+    [0, win_lengths[b]), stored as given (no quantization), and each query row
+    takes one softmax over all of them -- softmax(QK^T/sqrt(d))V over the
+    concatenation ("给长前缀列一张有单位的资源账本", section
+    "FlashAttention为什么不必保存整张热图": positions past either length take
+    no part).  GQA as in ``attend_gqa``.
+
+    q [B, H_q, Lq, D]; k_hat, v_hat [B, H_kv, N, D] decoded; k_win, v_win
+    [B, H_kv, W, D]; returns float64 [B, H_q, Lq, D].
+    """
+    b_, hq, lq, d = q.shape
+    hkv = k_hat.shape[1]
+    if hq % hkv:
+        raise ValueError("H_q must be a multiple of H_kv")
+    grp = hq // hkv
+    out = np.zeros((b_, hq, lq, v_hat.shape[-1]), np.float64)
+    for b in range(b_):
+        n, w = int(lengths[b]), int(win_lengths[b])
+        if n + w <= 0:
+            raise ValueError("a row with no valid key has no softmax")
+        for h in range(hq):
+            g = h // grp
+            k = np.concatenate([np.asarray(k_hat[b, g, :n], np.float64), np.asarray(k_win[b, g, :w], np.float64)])
+            v = np.concatenate([np.asarray(v_hat[b, g, :n], np.float64), np.asarray(v_win[b, g, :w], np.float64)])
+            out[b, h] = attend_dense(q[b, h], k, v, scale)
+    return out
+
+
 def rel_l2_error(out: np.ndarray, ref: np.ndarray) -> float:
     """||out - ref||_2 / ||ref||_2 over the whole output ("KV分组打包", section
     "同一输入上的精度与空间交换": relative L2 output error per input, then the

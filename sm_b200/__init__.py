@@ -21,6 +21,7 @@ import torch
 __all__ = [
     "KVQError", "PackedCache", "pack", "attend", "workspace_size", "check",
     "launch_count", "kernel_name", "cache_sizes", "lib", "LIB_PATH", "attend_noalloc",
+    "attend_window", "workspace_size_window",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
@@ -52,7 +53,7 @@ class _Cache(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libkvq.so not built: run `python -m sm_b200.build` ({LIB_PATH})")
+        raise ImportError(f"libkvq.so not built: run `python sm_b200/build.py` ({LIB_PATH})")
     L = ctypes.CDLL(LIB_PATH)
     i32, vp, sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
     L.kvq_cache_sizes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]
@@ -77,6 +78,11 @@ def _load() -> ctypes.CDLL:
     L.kvq_attend_noalloc.restype = ctypes.c_int
     L.kvq_noalloc_scratch_bytes.argtypes = []
     L.kvq_noalloc_scratch_bytes.restype = sz
+    L.kvq_attend_window.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, vp, vp, ctypes.c_int,
+                                    vp, i32, i32, i32, ctypes.c_float, vp, vp, sz, i32, vp]
+    L.kvq_attend_window.restype = ctypes.c_int
+    L.kvq_workspace_size_window.argtypes = [ctypes.POINTER(_Cache), i32, i32, i32]
+    L.kvq_workspace_size_window.restype = sz
     return L
 
 
@@ -248,6 +254,52 @@ def attend_noalloc(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, s
     _ok(lib.kvq_attend_noalloc(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(),
                                int(Q.shape[1]), int(Q.shape[2]), float(scale), out.data_ptr(),
                                int(splits), _stream(cache.device)), "kvq_attend_noalloc")
+    return out
+
+
+def workspace_size_window(cache: PackedCache, H_q: int, Lq: int, splits: int = 0) -> int:
+    c = cache.struct()
+    return int(lib.kvq_workspace_size_window(ctypes.byref(c), int(H_q), int(Lq), int(splits)))
+
+
+def attend_window(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, K_win: torch.Tensor,
+                  V_win: torch.Tensor, win_lengths: torch.Tensor, scale: float,
+                  out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                  splits: int = 0) -> torch.Tensor:
+    """Attention over the packed cache followed by a window of recent tokens
+    kept unquantized: sequence b's keys are its packed tokens [0, lengths[b])
+    then its window tokens [0, win_lengths[b]).  K_win, V_win
+    [B, H_kv, W_cap, D] fp32/bf16 (contiguous); lengths, win_lengths int32 [B]
+    on the device; returns O like Q."""
+    _check_cuda(Q, "Q", cache.device)
+    for t, n in ((lengths, "lengths"), (win_lengths, "win_lengths")):
+        _check_cuda(t, n, cache.device)
+        if t.dtype != torch.int32 or t.numel() != cache.B:
+            raise ValueError(f"{n} must be int32 [B]")
+    if Q.dim() != 4 or Q.shape[0] != cache.B or Q.shape[3] != cache.D:
+        raise ValueError("Q must be [B, H_q, Lq, D]")
+    for t, n in ((K_win, "K_win"), (V_win, "V_win")):
+        _check_cuda(t, n, cache.device)
+        if t.dim() != 4 or t.shape[0] != cache.B or t.shape[1] != cache.H_kv or t.shape[3] != cache.D:
+            raise ValueError(f"{n} must be [B, H_kv, W_cap, D]")
+    if K_win.shape != V_win.shape or K_win.dtype != V_win.dtype:
+        raise ValueError("K_win and V_win must match")
+    H_q, Lq, W_cap = int(Q.shape[1]), int(Q.shape[2]), int(K_win.shape[2])
+    if out is None:
+        out = torch.empty_like(Q)
+    else:
+        _check_cuda(out, "out", cache.device)
+        if out.shape != Q.shape or out.dtype != Q.dtype:
+            raise ValueError("out must match Q")
+    need = workspace_size_window(cache, H_q, Lq, splits)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=cache.device)
+    c = cache.struct()
+    _ok(lib.kvq_attend_window(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(),
+                              K_win.data_ptr(), V_win.data_ptr(), _dtype_code(K_win), win_lengths.data_ptr(),
+                              W_cap, H_q, Lq, float(scale), out.data_ptr(), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), int(splits),
+                              _stream(cache.device)), "kvq_attend_window")
     return out
 
 

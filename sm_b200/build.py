@@ -1,6 +1,6 @@
 """Build libkvq.so in-tree for sm_100a with nvcc.
 
-    python -m sm_b200.build [--force] [--verbose]
+    python sm_b200/build.py [--force] [--verbose]
 
 Every ``csrc/*.cu`` file compiles to an object under ``_build/`` (in
 parallel), and the objects link into ``sm_b200/libkvq.so``.  A source or

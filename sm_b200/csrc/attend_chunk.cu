@@ -106,6 +106,7 @@ struct ChunkParams {
   __nv_bfloat16* O;
   float* partials;                       // [slots][kD + 2][R]: m, z, u (feature-major)
   int ctas;
+  int force_partial;                     // a window follows: no CTA writes output rows
   unsigned int* err;
 };
 
@@ -332,8 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + kOffMisc);
 
   // sequences with a length outside 1..N_cap: report; rows of sequences with
-  // no valid key are zero (no block of theirs exists)
-  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+  // no valid key are zero (no block of theirs exists).  With a window the
+  // merge owns both.
+  for (int b = p.force_partial ? p.B : blockIdx.x; b < p.B; b += gridDim.x) {
     const int raw = p.lengths[b];
     if (threadIdx.x == 0 && (raw < 1 || raw > p.N_cap)) record_error(p.err, KVQ_ERR_LENGTH);
     if (slen[b] == 0) {
@@ -602,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             // the segment's last P V product must be done before O is read
             wait_bar(bar(PV_DONE + tile), k & 1u, p.err, abort_flag);
             tc_fence_after();
-            const bool whole = (c.seg.jb == 0) && (c.seg.je == c.seg.nb);
+            const bool whole = (c.seg.jb == 0) && (c.seg.je == c.seg.nb) && !p.force_partial;
             const long long head = static_cast<long long>(c.seg.b) * H + c.seg.h;
             const long long row = (static_cast<long long>(c.seg.b) * H * p.G + static_cast<long long>(c.seg.h) * p.G) *
                                       p.Lq + tile * 128 + r;
@@ -666,7 +668,8 @@ int chunk_ctas(const AttendArgs& a) {
 }
 
 size_t chunk_workspace(const AttendArgs& a) {
-  return partial_slots(chunk_ctas(a), a.g.B, a.g.H_kv) * rows_per_head(a) * (kD + 2) * sizeof(float);
+  return with_window_slots(a, partial_slots(chunk_ctas(a), a.g.B, a.g.H_kv),
+                           static_cast<size_t>(rows_per_head(a)) * (kD + 2) * sizeof(float));
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
@@ -731,6 +734,7 @@ kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   p.O = static_cast<__nv_bfloat16*>(a.O);
   p.partials = static_cast<float*>(a.workspace);
   p.ctas = ctas;
+  p.force_partial = a.win_lengths != nullptr;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
   if (launch_pdl(chunk_kernel, dim3(ctas), dim3(kThreads), smem, s, qmap, p) != cudaSuccess) return KVQ_ERR_CUDA;
@@ -752,6 +756,9 @@ kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   m.G = p.G;
   m.Lq = a.Lq;
   m.feature_major = true;
+  const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(ctas, a.g.B, a.g.H_kv)),
+                                   static_cast<long long>(kD + 2) * p.R, 1, p.R, &m, s);
+  if (ws != KVQ_OK) return ws;
   return launch_merge(m, s);
 }
 

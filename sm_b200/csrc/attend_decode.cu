@@ -10,25 +10,25 @@
 //
 // Layout of the work
 // ------------------
-// * Two CTAs per SM.  A CTA owns an equal share of the concatenated
-//   (b, h, 32-token block) list; a 32-token block is exactly one K group, so
-//   one K scale row serves the whole block.
-// * A CTA holds kNP warp pairs.  Each pair runs one 3-stage pipeline of bulk
-//   copies (cp.async.bulk, completion counted on an mbarrier) carrying, per
-//   block, 32 tokens of K codes (2 KB) and V codes (2 KB), the block's K
-//   scale row (512 B) and the tokens' V scales (512 B).
-//   - The S-warp (scores) folds the K scales into q once per block, unpacks
-//     K once for all four heads, sums lane partials through shared memory,
-//     runs the online softmax (m, z) and hands the V-warp each token's
-//     probabilities already multiplied by the token's V scales.  Scores are
-//     in log2 units (q carries scale * log2(e)), so exp is one ex2.
-//   - The V-warp (values) rescales its accumulators when m grows and adds
-//     p' * v for its 16 channels and four heads with packed f32x2 FMAs.
-//   Splitting the roles keeps each warp under 128 registers, so an SM runs
-//   16 warps.
-// * At the end of each (b, h) segment the pair states are merged in shared
-//   memory with the same rule and written as the output (segment covered
-//   whole by the CTA) or as a partial for the split merge kernel.
+// * The concatenated (b, h, 32-token block) list is split evenly over
+//   workers, one worker per warp pair (CTAs x pairs per CTA), each with a
+//   contiguous range; a 32-token block is exactly one K group, so one K scale
+//   row serves the whole block.  After the prologue no barrier spans more
+//   than a pair: every pair runs at its own pace.
+// * Each pair runs one pipeline of bulk copies (cp.async.bulk, completion
+//   counted on an mbarrier) carrying, per block, 32 tokens of K codes and V
+//   codes, the block's K scale row (512 B) and the tokens' V scales (512 B).
+//   - The S-warp (scores) keeps the segment's q in shared memory, folds the
+//     K scales into it once per block, unpacks K once for all four heads and
+//     writes per-lane partial scores; it also refills the pipeline.
+//   - The V-warp (values) sums the partials into scores, runs the online
+//     softmax (m, z) in log2 units (q carries scale * log2(e), so exp is one
+//     ex2), rescales its accumulators when m grows and adds p * s_v * v for
+//     its 16 channels and four heads with packed f32x2 FMAs.
+//   Splitting the roles keeps each warp at 128 registers.
+// * At the end of each (b, h) segment of its range the V-warp writes the
+//   pair's state: the output if the range covered the segment whole, else a
+//   partial (m, z, u) for the split merge kernel.
 //
 // Unpacking without a subtract
 // ----------------------------
@@ -51,13 +51,16 @@ namespace {
 constexpr int kD = 128;
 constexpr int kG = 4;                 // query heads per KV head
 constexpr int kTB = 32;               // tokens per block (one K group)
-// Per code width: warp pairs per CTA, pipeline stages per pair, code bytes
-// per token.  8-bit blocks carry twice the code bytes, so a CTA runs three
-// pairs of two stages to keep two CTAs on an SM.
+// Per code width: warp pairs per CTA, CTAs per SM, pipeline stages per pair,
+// code bytes per token.  4-bit: one CTA of eight pairs (three stages each)
+// per SM, which measured a little faster than two CTAs of four: co-resident
+// CTAs are not scheduled evenly, and the one the SM favours finishes well
+// before the other.  8-bit blocks carry twice the code bytes, so a CTA runs
+// three pairs of two stages and two CTAs share an SM.
 template <int BITS>
 struct Tr {
-  static constexpr int kNP = BITS == 4 ? 4 : 3;
-  static constexpr int kCtasPerSm = 2;
+  static constexpr int kNP = BITS == 4 ? 8 : 3;
+  static constexpr int kCtasPerSm = BITS == 4 ? 1 : 2;
   static constexpr int kS = BITS == 4 ? 3 : 2;
   static constexpr int kThreads = 2 * kNP * 32;
   static constexpr int kCb = BITS == 4 ? 64 : 128;
@@ -111,6 +114,7 @@ struct DecodeParams {
   void* O;
   float* partials;                    // [slots][kG][kD + 2]
   int ctas;                           // CTAs; each warp pair is one worker of the plan
+  int force_partial;                  // a window follows: no worker writes output rows
   unsigned int* err;
 };
 
@@ -598,7 +602,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) z[hh] += __shfl_xor_sync(0xffffffffu, z[hh], o);
       }
-      const bool whole = (seg.jb == 0) && (seg.je == seg.nb);
+      const bool whole = (seg.jb == 0) && (seg.je == seg.nb) && !p.force_partial;
       const long long slot = static_cast<long long>(worker) + head;
 #pragma unroll
       for (int hh = 0; hh < kG; ++hh) {
@@ -642,14 +646,15 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-// Shared memory one CTA may use so that Tr::kCtasPerSm of them fit an SM
-// (228 KB per SM, 1 KB of it reserved per CTA, at most 227 KB per CTA).
-constexpr size_t kSmemPerCta = 113 * 1024;
+// Shared memory one CTA may use so that `per_sm` of them fit an SM (228 KB
+// per SM, 1 KB of it reserved per CTA, at most 227 KB per CTA).
+constexpr size_t smem_limit(int per_sm) { return per_sm == 1 ? 227 * 1024 : 113 * 1024; }
 
 bool decode_applies(const AttendArgs& a) {
   return (a.g.bits == 4 || a.g.bits == 8) && a.g.group == kTB && a.g.D == kD && a.Lq == 1 &&
          a.H_q == kG * a.g.H_kv &&
-         (a.g.bits == 4 ? smem_bytes<4>(a.g.B) : smem_bytes<8>(a.g.B)) <= kSmemPerCta;
+         (a.g.bits == 4 ? smem_bytes<4>(a.g.B) <= smem_limit(Tr<4>::kCtasPerSm)
+                        : smem_bytes<8>(a.g.B) <= smem_limit(Tr<8>::kCtasPerSm));
 }
 
 int decode_ctas(const AttendArgs& a) {
@@ -665,7 +670,8 @@ int decode_ctas(const AttendArgs& a) {
 int decode_pairs(const AttendArgs& a) { return a.g.bits == 4 ? Tr<4>::kNP : Tr<8>::kNP; }
 
 size_t decode_workspace(const AttendArgs& a) {
-  return partial_slots(decode_ctas(a) * decode_pairs(a), a.g.B, a.g.H_kv) * kG * (kD + 2) * sizeof(float);
+  return with_window_slots(a, partial_slots(decode_ctas(a) * decode_pairs(a), a.g.B, a.g.H_kv),
+                           kG * (kD + 2) * sizeof(float));
 }
 
 kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
@@ -696,6 +702,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   p.O = a.O;
   p.partials = static_cast<float*>(a.workspace);
   p.ctas = ctas;
+  p.force_partial = a.win_lengths != nullptr;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
   const cudaError_t le = launch_pdl(kernel, dim3(ctas), dim3(threads), smem, s, p);
@@ -717,6 +724,9 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   m.D = kD;
   m.G = kG;
   m.Lq = 1;
+  const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(m.ctas, a.g.B, a.g.H_kv)),
+                                   kG * (kD + 2), kD + 2, 1, &m, s);
+  if (ws != KVQ_OK) return ws;
   return launch_merge(m, s);
 }
 

@@ -34,6 +34,7 @@ struct GenericParams {
   void* O;
   float* partials;             // [slots][n_rt*kRT][D + 2]
   int ctas;
+  int force_partial;           // a window follows: no CTA writes output rows
 };
 
 __device__ __forceinline__ int code_at(const uint8_t* codes, long long flat, int bits) {
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kThreads) attend_generic_kernel(GenericParams 
     const int len = clamp_len(p.lengths[b], p.N_cap);
     const int j_begin = j;
     const int j_end = static_cast<int>(min(static_cast<long long>(nb), j + (cr.g1 - g)));
-    const bool whole = (j_begin == 0) && (j_end == nb);
+    const bool whole = (j_begin == 0) && (j_end == nb) && !p.force_partial;
     const long long head = static_cast<long long>(b) * H + h;
     const long long row_base = (static_cast<long long>(b) * H * p.G + static_cast<long long>(h) * p.G) * p.Lq + r0;
     const uint8_t* kc = p.k_codes + head * p.k_codes_head;
@@ -205,7 +206,8 @@ bool generic_applies(const AttendArgs& a) { return a.g.D <= 256; }
 size_t generic_workspace(const AttendArgs& a) {
   const int R = rows_per_head(a);
   const int n_rt = (R + kRT - 1) / kRT;
-  return partial_slots(generic_ctas(a), a.g.B, a.g.H_kv) * n_rt * kRT * (a.g.D + 2) * sizeof(float);
+  return with_window_slots(a, partial_slots(generic_ctas(a), a.g.B, a.g.H_kv),
+                           static_cast<size_t>(n_rt) * kRT * (a.g.D + 2) * sizeof(float));
 }
 
 kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
@@ -245,6 +247,7 @@ kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
   p.O = a.O;
   p.partials = static_cast<float*>(a.workspace);
   p.ctas = ctas;
+  p.force_partial = a.win_lengths != nullptr;
   const cudaError_t le = launch_pdl(attend_generic_kernel, dim3(ctas, n_rt), dim3(kThreads), smem, s, p);
   if (le != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
@@ -264,6 +267,9 @@ kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
   m.D = a.g.D;
   m.G = p.G;
   m.Lq = a.Lq;
+  const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(ctas, a.g.B, a.g.H_kv)),
+                                   static_cast<long long>(n_rt) * kRT * (a.g.D + 2), a.g.D + 2, 1, &m, s);
+  if (ws != KVQ_OK) return ws;
   return launch_merge(m, s);
 }
 

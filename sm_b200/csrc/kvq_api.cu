@@ -187,6 +187,60 @@ kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
   return impl.launch(a, static_cast<cudaStream_t>(stream));
 }
 
+static bool fill_window(const void* K_win, const void* V_win, kvq_dtype win_dtype,
+                        const int32_t* win_lengths, int32_t W_cap, AttendArgs* a) {
+  if (win_dtype != KVQ_F32 && win_dtype != KVQ_BF16) return false;
+  if (W_cap < 1) return false;
+  a->K_win = K_win;
+  a->V_win = V_win;
+  a->win_dtype = win_dtype;
+  a->win_lengths = win_lengths;
+  a->W_cap = W_cap;
+  return true;
+}
+
+size_t kvq_workspace_size_window(const kvq_cache* cache, int32_t H_q, int32_t Lq, int32_t splits) {
+  AttendArgs a{};
+  if (!fill_attend_args(nullptr, KVQ_BF16, cache, nullptr, H_q, Lq, 1.f, nullptr, nullptr, 0,
+                        splits, &a))
+    return 0;
+  static const int32_t dummy = 0;
+  a.win_lengths = &dummy;                // only "has a window" matters for the size
+  a.W_cap = 1;
+  const AttendImpl& impl = choose(a);
+  return impl.workspace(a);
+}
+
+kvq_status kvq_attend_window(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                             const int32_t* lengths, const void* K_win, const void* V_win,
+                             kvq_dtype win_dtype, const int32_t* win_lengths, int32_t W_cap,
+                             int32_t H_q, int32_t Lq, float scale, void* O, void* workspace,
+                             size_t ws_bytes, int32_t splits, void* stream) {
+  AttendArgs a{};
+  if (!fill_attend_args(Q, q_dtype, cache, lengths, H_q, Lq, scale, O, workspace, ws_bytes,
+                        splits, &a))
+    return KVQ_ERR_ARG;
+  if (!fill_window(K_win, V_win, win_dtype, win_lengths, W_cap, &a)) return KVQ_ERR_ARG;
+  if (!Q || !O || !lengths || !K_win || !V_win || !win_lengths || !cache->k_codes || !cache->k_scales ||
+      !cache->v_codes || !cache->v_scales)
+    return KVQ_ERR_ARG;
+  if (cache->D > 256) return KVQ_ERR_UNSUPPORTED;
+  if (cache->B > 8192) return KVQ_ERR_UNSUPPORTED;
+  if (!aligned16(cache->k_codes) || !aligned16(cache->k_scales) || !aligned16(cache->v_codes) ||
+      !aligned16(cache->v_scales))
+    return KVQ_ERR_ALIGN;
+  const size_t esz = q_dtype == KVQ_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) % esz) return KVQ_ERR_ALIGN;
+  const size_t wsz = win_dtype == KVQ_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(K_win) | reinterpret_cast<uintptr_t>(V_win)) % wsz) return KVQ_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(lengths) | reinterpret_cast<uintptr_t>(win_lengths)) % 4) return KVQ_ERR_ALIGN;
+  const AttendImpl& impl = choose(a);
+  const size_t need = impl.workspace(a);
+  if (!workspace || ws_bytes < need) return KVQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
+  return impl.launch(a, static_cast<cudaStream_t>(stream));
+}
+
 kvq_status kvq_check(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned int h = 0;

@@ -114,8 +114,41 @@ struct MergeArgs {
   int R, R_pad, D;                 // rows per (b,h) and the padded row count of a slot
   int G, Lq;                       // query heads per KV head, rows per query head
   bool feature_major;              // partial layout (rows contiguous per field)
+  // recent-token window (kvq_attend_window); win_lengths == nullptr: none.
+  // With a window every (b, h) is merged: its window state sits in slot
+  // win_slot0 + b * H_kv + h, and no worker wrote an output row itself.
+  const int32_t* win_lengths;
+  int W_cap;
+  long long win_slot0;
 };
 kvq_status launch_merge(const MergeArgs& a, cudaStream_t s);
+
+// The window's partial state (m, z, u) of every row of every (b, h), written
+// into slot slot0 + b * H_kv + h of the caller's partial layout: element
+// (row r, field f) of a slot at r * row_stride + f * field_stride (field 0 =
+// m in natural-log units, 1 = z, 2 + d = u[d]).
+struct WindowArgs {
+  const void* Q;
+  int q_dtype;
+  const void* K_win;
+  const void* V_win;
+  int win_dtype;
+  const int32_t* win_lengths;
+  int W_cap;
+  int B, H_kv, G, Lq, D;
+  float scale;
+  float* partials;
+  long long slot0, slot_stride, row_stride, field_stride;
+};
+kvq_status launch_window(const WindowArgs& w, cudaStream_t s);
+
+struct AttendArgs;
+// After an implementation's packed-cache kernel: when the call has a window,
+// launch the window kernel into slots [slot0, slot0 + B * H_kv) of
+// `partials` (laid out with the given strides, in floats) and point the
+// merge at them.  Without a window it does nothing.
+kvq_status add_window(const AttendArgs& a, float* partials, long long slot0, long long slot_stride,
+                      long long row_stride, long long field_stride, MergeArgs* m, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // kernels' host launchers
@@ -148,7 +181,20 @@ struct AttendArgs {
   void* workspace;
   size_t ws_bytes;
   int splits;
+  // recent-token window (kvq_attend_window); win_lengths == nullptr: none
+  const void* K_win;
+  const void* V_win;
+  int win_dtype;
+  const int32_t* win_lengths;
+  int W_cap;
 };
+
+// Workspace of an implementation whose packed partials fill `slots` slots of
+// `slot_bytes`: a window adds one slot per (b, h) after them.
+inline size_t with_window_slots(const AttendArgs& a, size_t slots, size_t slot_bytes) {
+  const size_t win = a.win_lengths ? static_cast<size_t>(a.g.B) * static_cast<size_t>(a.g.H_kv) : 0;
+  return (slots + win) * slot_bytes;
+}
 
 // One implementation of kvq_attend: how much workspace it needs and how to
 // launch it.  `applies` says whether it handles these arguments.

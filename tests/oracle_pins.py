@@ -325,6 +325,40 @@ def pin_gqa_and_lengths():
             assert np.max(np.abs(out[b, h] - bf)) < 1e-12
 
 
+def pin_window():
+    """Packed cache plus an unquantized recent window: brute force over the
+    concatenated keys of each (b, head), window positions past each
+    sequence's window length ignored (filled with huge values here so that
+    reading them would show), a packed part of length 0, and the two-part
+    block merge of the packed and window states giving the same rows."""
+    rng = np.random.default_rng(21)
+    b_, hq, hkv, lq, n, w_cap, d = 3, 4, 2, 2, 7, 5, 6
+    q = rng.standard_normal((b_, hq, lq, d))
+    k = rng.standard_normal((b_, hkv, n, d))
+    v = rng.standard_normal((b_, hkv, n, d))
+    kw = rng.standard_normal((b_, hkv, w_cap, d))
+    vw = rng.standard_normal((b_, hkv, w_cap, d))
+    lens, wl = [7, 0, 3], [2, 5, 0]
+    for b in range(b_):
+        kw[b, :, wl[b]:] = 1e6
+        vw[b, :, wl[b]:] = -1e6
+    out = O.attend_gqa_window(q, k, v, lens, kw, vw, wl, 0.7)
+    for b in range(b_):
+        for h in range(hq):
+            hk = h // (hq // hkv)
+            kk = np.concatenate([k[b, hk, :lens[b]], kw[b, hk, :wl[b]]])
+            vv = np.concatenate([v[b, hk, :lens[b]], vw[b, hk, :wl[b]]])
+            bf = O.attend_bruteforce(q[b, h], kk, vv, 0.7)
+            assert np.max(np.abs(out[b, h] - bf)) < 1e-12
+            if lens[b] and wl[b]:
+                st = O.merge_partials(O.partial_state(q[b, h], k[b, hk, :lens[b]], v[b, hk, :lens[b]], 0.7),
+                                      O.partial_state(q[b, h], kw[b, hk, :wl[b]], vw[b, hk, :wl[b]], 0.7))
+                assert np.max(np.abs(st[2] / st[1][:, None] - out[b, h])) < 1e-12
+    # no window at all is the plain cache
+    assert np.max(np.abs(O.attend_gqa_window(q, k, v, [7, 4, 3], kw, vw, [0, 0, 0], 0.7)
+                         - O.attend_gqa(q, k, v, [7, 4, 3], 0.7))) < 1e-12
+
+
 def pin_rel_l2_band():
     """Soft check (parity unpinned at the value level): the mean relative L2
     output error on the six clean inputs lands near the pages' table, and the
@@ -352,5 +386,5 @@ ALL_PINS = [
     pin_error_bound, pin_grouping_axes, pin_flat_pairing_odd_width, pin_crop_35x13,
     pin_eight_bit, pin_ledger, pin_workspace_sizes, pin_17_over_3,
     pin_negative_example, pin_dense_vs_blocked, pin_bruteforce,
-    pin_large_scores_stay_finite, pin_merge_partials, pin_gqa_and_lengths,
+    pin_large_scores_stay_finite, pin_merge_partials, pin_gqa_and_lengths, pin_window,
 ]

@@ -150,6 +150,25 @@ def _dense_without_scale(q, k, v, scale):
     return (w @ v) / w.sum(axis=1, keepdims=True)
 
 
+def _window_scale_dropped(q, k_hat, v_hat, lengths, k_win, v_win, win_lengths, scale):
+    out = _ORIG_WINDOW(q, k_hat, v_hat, lengths, k_win, v_win, win_lengths, 1.0)
+    return out
+
+
+def _window_length_ignored(q, k_hat, v_hat, lengths, k_win, v_win, win_lengths, scale):
+    full = [k_win.shape[2]] * len(win_lengths)
+    return _ORIG_WINDOW(q, k_hat, v_hat, lengths, k_win, v_win, full, scale)
+
+
+def _window_before_packed_length(q, k_hat, v_hat, lengths, k_win, v_win, win_lengths, scale):
+    # the window replaces the packed tail instead of following it
+    cut = [max(0, int(n) - int(w)) for n, w in zip(lengths, win_lengths)]
+    return _ORIG_WINDOW(q, k_hat, v_hat, cut, k_win, v_win, win_lengths, scale)
+
+
+_ORIG_WINDOW = O.attend_gqa_window
+
+
 MUTATIONS = {
     "nibble_order_swapped": [("pair_nibbles", _swapped_pair), ("split_nibbles", _swapped_split)],
     "round_half_up": [("quantize_groups", _round_half_up)],
@@ -164,6 +183,9 @@ MUTATIONS = {
     "decode_keeps_padding": [("unpack_matrix", _unpack_no_crop)],
     "score_scale_dropped": [("attend_dense", _dense_without_scale)],
     "eight_bit_bias_128": [("QMAX", {4: 7, 8: 128})],
+    "window_scale_dropped": [("attend_gqa_window", _window_scale_dropped)],
+    "window_length_ignored": [("attend_gqa_window", _window_length_ignored)],
+    "window_replaces_packed_tail": [("attend_gqa_window", _window_before_packed_length)],
 }
 
 

@@ -335,3 +335,119 @@ def test_long_context_full(sm):
 @pytest.mark.parametrize("bits", [4, 8])
 def test_chunk_full(sm, bits):
     _full_case(sm, "chunk", bits=bits, heads=[(0, 0), (1, 5), (3, 7)])
+
+
+# ---------------------------------------------------------------------------
+# attend with a recent-token window kept unquantized (kvq_attend_window)
+# ---------------------------------------------------------------------------
+
+def _check_window(sm, q, k, v, lens, kw, vw, wl, bits, group, scale, q_dtype=torch.bfloat16,
+                  win_dtype=torch.float32, splits=0):
+    """kvq_attend_window against the oracle's softmax over the decoded packed
+    tokens followed by the window tokens (as stored, bf16-rounded where the
+    window is bf16), within 2e-3 * max|V| over the values attended."""
+    b_, hq, lq, d = q.shape
+    hkv = k.shape[1]
+    cache = pack_gpu(sm, k, v, bits, group)
+    qd = to_dev(q, q_dtype)
+    kwd, vwd = to_dev(kw, win_dtype), to_dev(vw, win_dtype)
+    out = sm.attend_window(qd, cache, to_dev(lens, torch.int32), kwd, vwd, to_dev(wl, torch.int32), scale,
+                           splits=splits)
+    sm.check()
+    assert out.dtype == q_dtype
+    o = out.float().cpu().numpy()
+    k_hat, v_hat = np.zeros_like(k), np.zeros_like(v)
+    for b in range(b_):
+        for h in range(hkv):
+            k_hat[b, h] = O.unpack_matrix(O.pack_k(k[b, h], bits, group))
+            v_hat[b, h] = O.unpack_matrix(O.pack_v(v[b, h], bits, group))
+    kwv, vwv = kwd.float().cpu().numpy(), vwd.float().cpu().numpy()
+    want = O.attend_gqa_window(qd.float().cpu().numpy(), k_hat, v_hat, lens, kwv, vwv, wl, scale)
+    for b in range(b_):
+        vals = np.concatenate([v_hat[b, :, :lens[b]].ravel(), vwv[b, :, :wl[b]].ravel()])
+        tol = 2e-3 * float(np.abs(vals).max())
+        # a bf16 output carries its own rounding, up to 2^-8 of the value: a
+        # row that follows one window key can sit near max|V| itself
+        err = np.abs(o[b] - want[b])
+        if q_dtype == torch.bfloat16:
+            err = err - np.abs(want[b]) * 2.0 ** -8
+        worst = float(err.max())
+        assert np.isfinite(o[b]).all() and worst <= tol, f"b{b}: max|err| {worst:.3e} > {tol:.3e}"
+    return o
+
+
+def _window(b_, hkv, w_cap, d, wl, seed):
+    rng = np.random.default_rng(seed)
+    kw = rng.standard_normal((b_, hkv, w_cap, d)).astype(np.float32)
+    vw = rng.standard_normal((b_, hkv, w_cap, d)).astype(np.float32)
+    wl = np.asarray(wl, np.int32)
+    for b in range(b_):
+        kw[b, :, wl[b]:] = 1e4          # past a window's length: must not be read
+        vw[b, :, wl[b]:] = -1e4
+    return kw, vw, wl
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("win_dtype", [torch.float32, torch.bfloat16])
+def test_window_decode(sm, bits, win_dtype):
+    """Tuned decode kernel (four heads per KV head, D 128, g 32) plus a
+    window: packed lengths ending inside a block, one sequence with no packed
+    token (window only), one with an empty window, several splits."""
+    q, k, v, lens = _gqa_case(4, 8, 2, 700, 128, [700, 0, 300, 29], seed=60 + bits, bits=bits, outliers=True)
+    cache = pack_gpu(sm, k, v, bits, 32)
+    assert sm.kernel_name(cache, 8, 1).startswith("decode_gqa4")
+    kw, vw, wl = _window(4, 2, 32, 128, [31, 5, 0, 32], seed=61)
+    for splits in (0, 1, 5):
+        _check_window(sm, q, k, v, lens, kw, vw, wl, bits, 32, 1.0, win_dtype=win_dtype, splits=splits)
+
+
+def test_window_decode_long(sm):
+    """A long sequence split over many workers (the part-parallel merge) plus
+    a window whose keys dominate some rows (large scores)."""
+    q, k, v, lens = _gqa_case(1, 8, 2, 20000, 128, [19999], seed=62)
+    kw, vw, wl = _window(1, 2, 64, 128, [40], seed=63)
+    kw[:, :, :8] *= 4.0
+    _check_window(sm, q, k, v, lens, kw, vw, wl, 4, 32, 1.0)
+
+
+@pytest.mark.parametrize("lq", [32, 64])
+def test_window_chunk(sm, lq):
+    """Tensor-core chunk kernel (feature-major partials) plus a window."""
+    q, k, v, lens = _gqa_case(3, 8, 2, 700, 128, [700, 300, 0], lq=lq, seed=64)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    assert sm.kernel_name(cache, 8, lq).startswith("chunk")
+    kw, vw, wl = _window(3, 2, 48, 128, [48, 0, 7], seed=65)
+    for splits in (0, 1):
+        _check_window(sm, q, k, v, lens, kw, vw, wl, 4, 32, 1.0, splits=splits)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 8), (8, 32)])
+def test_window_generic(sm, bits, group):
+    """Generic kernel (D 64, several query rows) plus a window, f32 Q."""
+    q, k, v, lens = _gqa_case(3, 4, 2, 200, 64, [200, 1, 0], lq=3, seed=66, bits=bits, group=group)
+    kw, vw, wl = _window(3, 2, 20, 64, [3, 20, 1], seed=67)
+    _check_window(sm, q, k, v, lens, kw, vw, wl, bits, group, 0.125, q_dtype=torch.float32)
+
+
+def test_window_bad_lengths(sm):
+    """No key at all (both lengths 0) or a window length past its capacity is
+    reported; the keyless sequence's rows are zeros, the others stay finite."""
+    q, k, v, _ = _gqa_case(3, 8, 2, 256, 128, [256, 256, 256], seed=68)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    kw, vw, _ = _window(3, 2, 16, 128, [16, 16, 16], seed=69)
+    out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+    lens = torch.tensor([256, 0, 100], dtype=torch.int32, device=DEV)
+    wl = torch.tensor([3, 0, 16], dtype=torch.int32, device=DEV)
+    sm.attend_window(to_dev(q, torch.bfloat16), cache, lens, to_dev(kw), to_dev(vw), wl, 1.0, out=out)
+    with pytest.raises(sm.KVQError) as e:
+        sm.check()
+    assert e.value.name == "KVQ_ERR_LENGTH"
+    assert torch.all(out[1] == 0)
+    assert torch.isfinite(out.float()).all()
+    sm.check()
+    wl = torch.tensor([3, 17, 16], dtype=torch.int32, device=DEV)
+    lens = torch.tensor([256, 10, 100], dtype=torch.int32, device=DEV)
+    sm.attend_window(to_dev(q, torch.bfloat16), cache, lens, to_dev(kw), to_dev(vw), wl, 1.0, out=out)
+    with pytest.raises(sm.KVQError):
+        sm.check()
+    sm.check()
