@@ -123,18 +123,20 @@ def measured_peaks(kind: str = "hbm"):
 
 
 PROFILE_FOR = {
-    ("decode_gqa", 4): "attend_decode_gqa_b32_ctx4096.md",
-    ("decode_gqa", 8): "attend_decode_gqa_b32_ctx4096_8bit.md",
-    ("chunk", 4): "attend_chunk_b4_lq64_ctx16384.md",
+    ("decode_gqa", 4, 32): "attend_decode_gqa_b32_ctx4096.md",
+    ("decode_gqa", 8, 32): "attend_decode_gqa_b32_ctx4096_8bit.md",
+    ("chunk", 4, 32): "attend_chunk_b4_lq64_ctx16384.md",
 }
 
 
-def recorded_traffic(kernel_src: str, workload: str = "decode_gqa", bits: int = 4):
+def recorded_traffic(kernel_src: str, workload: str = "decode_gqa", bits: int = 4, group: int = 32,
+                     window: int = 0):
     """Per-launch DRAM bytes of the attend kernel from the committed ncu
-    summary of this workload and code width, or None when there is none or
-    the kernel source changed since the capture."""
+    summary of this workload, code width and group size, or None when there
+    is none (a window is not profiled) or the kernel source changed since
+    the capture."""
     import hashlib
-    name = PROFILE_FOR.get((workload, bits))
+    name = None if window else PROFILE_FOR.get((workload, bits, group))
     if name is None:
         return None
     summary = os.path.join(ROOT, "profiles", name)
@@ -292,8 +294,14 @@ def run_kvq(args, rank, world, local_rank):
     B, H_q, H_kv, D, N, Lq = meta["B"], meta["H_q"], meta["H_kv"], meta["D"], meta["N"], meta["Lq"]
     bits = args.bits if args.bits else (meta["bits"] if isinstance(meta["bits"], int) else 4)
     meta["bits"] = bits
+    if args.group:
+        meta["group"] = args.group
     g = meta["group"]
     uniform = bool(np.all(lens_np == N))
+    # --window W: the last W tokens of each sequence stay unquantized (bf16)
+    # in a recent-token window; the packed cache holds the tokens before them
+    W_win = int(args.window)
+    append = uniform and not W_win
     # the step's append: the K group(s) holding the new tokens (re-packed from a
     # float32 recent-token window) and the new tokens' V rows; only when every
     # sequence has the same length, since one kvq_pack call covers one range
@@ -313,20 +321,41 @@ def run_kvq(args, rank, world, local_rank):
     qd = torch.from_numpy(q_np).to(dev).to(torch.bfloat16)
     lens = torch.from_numpy(lens_np).to(dev)
     out = torch.empty_like(qd)
-    ws_need = K.workspace_size(caches[0], H_q, Lq)
+    if W_win:
+        wl_np = np.minimum(lens_np, W_win).astype(np.int32)
+        lens_p_np = (lens_np - wl_np).astype(np.int32)
+        kw_np = np.zeros((B, H_kv, W_win, D), np.float32)
+        vw_np = np.zeros((B, H_kv, W_win, D), np.float32)
+        for b in range(B):
+            n, w = int(lens_np[b]), int(wl_np[b])
+            kw_np[b, :, :w] = k_np[b, :, n - w:n]
+            vw_np[b, :, :w] = v_np[b, :, n - w:n]
+        kwin = torch.from_numpy(kw_np).to(dev).to(torch.bfloat16)
+        vwin = torch.from_numpy(vw_np).to(dev).to(torch.bfloat16)
+        lens = torch.from_numpy(lens_p_np).to(dev)
+        wlens = torch.from_numpy(wl_np).to(dev)
+        ws_need = K.workspace_size_window(caches[0], H_q, Lq)
+    else:
+        ws_need = K.workspace_size(caches[0], H_q, Lq)
     ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
+
+    def attend_call(c):
+        if W_win:
+            K.attend_window(qd, c, lens, kwin, vwin, wlens, 1.0, out=out, workspace=ws)
+        else:
+            K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
     torch.cuda.synchronize()
     K.check(dev)
 
     def step(i):
         c = caches[i & 1]
-        if uniform:
+        if append:
             K.pack(win_k, None, c, t0=t0)
             K.pack(None, new_v, c, t0=v0)
-        K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
+        attend_call(c)
 
     def attend_only(i):
-        K.attend(qd, caches[i & 1], lens, 1.0, out=out, workspace=ws)
+        attend_call(caches[i & 1])
 
     stream = torch.cuda.current_stream(dev)
     for i in range(args.warmup):
@@ -399,21 +428,25 @@ def run_kvq(args, rank, world, local_rank):
     for i in range(args.steps):
         c = caches[i & 1]
         qd.copy_(q_host, non_blocking=True)
-        if uniform:
+        if append:
             win_k[:, :, -Lq:].copy_(kv_host_k, non_blocking=True)
             new_v.copy_(kv_host_v, non_blocking=True)
             K.pack(win_k, None, c, t0=t0)
             K.pack(None, new_v, c, t0=v0)
-        K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
+        attend_call(c)
         o_host.copy_(out, non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
-    h2d = q_host.numel() * 2 + ((kv_host_k.numel() + kv_host_v.numel()) * 4 if uniform else 0)
+    h2d = q_host.numel() * 2 + ((kv_host_k.numel() + kv_host_v.numel()) * 4 if append else 0)
     d2h = o_host.numel() * 2
 
-    abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g, lq=Lq)
-    step_bytes = abytes + (append_bytes(B, H_kv, D, N - t0, Lq, bits, g) if uniform else 0)
+    if W_win:
+        # packed tokens as usual plus the window's bf16 K and V rows
+        abytes = attend_bytes(B, H_q, H_kv, D, lens_p_np, bits, g, lq=Lq) + H_kv * D * 2 * 2 * int(np.sum(wl_np))
+    else:
+        abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g, lq=Lq)
+    step_bytes = abytes + (append_bytes(B, H_kv, D, N - t0, Lq, bits, g) if append else 0)
     attend_flops = 4 * H_q * Lq * D * int(np.sum(lens_np.astype(np.int64)))
     ms_max, e2e_max = max_over_ranks([ms, e2e_ms], world, dev)
 
@@ -445,7 +478,10 @@ def run_kvq(args, rank, world, local_rank):
                        "context": N if uniform else "per-sequence", "lengths_sum": int(np.sum(lens_np)),
                        "bits": bits, "group": g, "lq": Lq,
                        "step": ("append (re-pack the K group(s) of the new tokens, pack their V rows) + attend"
-                                if uniform else "attend (per-sequence lengths; no shared append range)"),
+                                if append else
+                                f"attend over the packed tokens and a {W_win}-token bf16 window" if W_win else
+                                "attend (per-sequence lengths; no shared append range)"),
+                       "window": W_win,
                        "l2": f"inputs larger than L2: 2 packed caches of {caches[0].nbytes() / 1e6:.0f} MB used in turn",
                        "parallelism": f"independent batch per GPU x{world}",
                        "attend_kernel": kname, "step_bytes": step_bytes,
@@ -460,7 +496,7 @@ def run_kvq(args, rank, world, local_rank):
                          "algorithmic_bytes_per_launch": abytes,
                          "algorithmic_flops_per_launch": attend_flops,
                          "attend_gbs": round(abytes / (att_ms * 1e-3) / 1e9, 1),
-                         "traffic": recorded_traffic(src, workload, bits)},
+                         "traffic": recorded_traffic(src, workload, bits, g, W_win)},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_max / args.steps * 1e3, 3)},
             "gpu_launches": int(launches),
@@ -483,6 +519,11 @@ def main():
                     help="the decode GQA workload is the headline; the others are for study")
     ap.add_argument("--bits", type=int, choices=[4, 8], default=0,
                     help="code width (default: the workload's, 4 for the chunk workload)")
+    ap.add_argument("--group", type=int, choices=[8, 32], default=0,
+                    help="scale group size (default: the workload's, 32)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="keep the last W tokens of each sequence unquantized (bf16) in a recent-token "
+                         "window (kvq_attend_window); 0 = none")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -497,8 +538,10 @@ def main():
         q, k, v, lens, meta = W.gqa_case(args.workload, SEED)
         import torch
         q = torch.from_numpy(q).to(torch.bfloat16).float().numpy()
-        if not isinstance(meta["bits"], int):
+        if args.bits or not isinstance(meta["bits"], int):
             meta["bits"] = args.bits or 4
+        if args.group:
+            meta["group"] = args.group
         per_step = max(4, args.cpu_heads // 4)
         total, times = 0, []
         for _ in range(args.warmup):
@@ -536,7 +579,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     res, data = run_kvq(args, rank, world, local_rank)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and not args.window:
         q, k, v, lens, meta = data
         nb, ts, heads = cpu_oracle_rate(q, k, v, lens, meta, args.cpu_heads, repeats=3, min_seconds=10.0)
         rate = nb / statistics.median(ts) / 1e9

@@ -51,19 +51,25 @@ namespace {
 constexpr int kD = 128;
 constexpr int kG = 4;                 // query heads per KV head
 constexpr int kTB = 32;               // tokens per block (one K group)
-// Per code width: warp pairs per CTA, CTAs per SM, pipeline stages per pair,
-// code bytes per token.  4-bit: one CTA of eight pairs (three stages each)
-// per SM, which measured a little faster than two CTAs of four: co-resident
-// CTAs are not scheduled evenly, and the one the SM favours finishes well
-// before the other.  8-bit blocks carry twice the code bytes, so a CTA runs
-// three pairs of two stages and two CTAs share an SM.
-template <int BITS>
+// Per code width and group size: warp pairs per CTA, CTAs per SM, pipeline
+// stages per pair, code bytes per token, scale layout.  4-bit g32: one CTA
+// of eight pairs (three stages each) per SM, which measured a little faster
+// than two CTAs of four: co-resident CTAs are not scheduled evenly, and the
+// one the SM favours finishes well before the other.  8-bit g32 blocks
+// carry twice the code bytes: three pairs of two stages, two CTAs per SM.
+// g8 blocks carry four K scale rows and sixteen V scales per token: two
+// stages, eight pairs (4-bit) or six (8-bit) in one CTA per SM.
+template <int BITS, int GRP>
 struct Tr {
-  static constexpr int kNP = BITS == 4 ? 8 : 3;
-  static constexpr int kCtasPerSm = BITS == 4 ? 1 : 2;
-  static constexpr int kS = BITS == 4 ? 3 : 2;
+  static_assert(GRP == 32 || GRP == 8, "group of 32 or 8 tokens / features");
+  static constexpr int kNP = BITS == 4 ? 8 : (GRP == 32 ? 3 : 6);
+  static constexpr int kCtasPerSm = (BITS == 8 && GRP == 32) ? 2 : 1;
+  static constexpr int kS = (BITS == 4 && GRP == 32) ? 3 : 2;
   static constexpr int kThreads = 2 * kNP * 32;
   static constexpr int kCb = BITS == 4 ? 64 : 128;
+  static constexpr int kKsRows = 32 / GRP;          // K scale rows (groups) per 32-token block
+  static constexpr int kVs = 128 / GRP;             // V scales per token
+  static constexpr int kPvW = GRP == 32 ? 20 : 4;   // floats per token row of the p table
   // each channel's code f = 1 + code * eps sits in mantissa bits 15.. (even
   // 4-bit channels, every 8-bit channel: eps = 2^-8) or 19.. (odd 4-bit
   // channels: eps = 2^-4); corr = 1 + qmax * eps
@@ -75,30 +81,35 @@ struct Tr {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int BITS>
+template <int BITS, int GRP>
 struct Stage {
-  uint8_t kc[kTB * Tr<BITS>::kCb];    // K codes, 64 or 128 B per token
-  uint8_t vc[kTB * Tr<BITS>::kCb];    // V codes
-  float ks[kD];                       // K scale row of the block's group
-  float vs[kTB][kD / 32];             // V scales, 4 per token
+  uint8_t kc[kTB * Tr<BITS, GRP>::kCb];    // K codes, 64 or 128 B per token
+  uint8_t vc[kTB * Tr<BITS, GRP>::kCb];    // V codes
+  float ks[Tr<BITS, GRP>::kKsRows][kD];    // K scale rows of the block's groups
+  float vs[kTB][Tr<BITS, GRP>::kVs];       // V scales, 4 (g32) or 16 (g8) per token
 };
 
-template <int BITS>
+template <int BITS, int GRP>
 struct PairSmem {
-  Stage<BITS> st[Tr<BITS>::kS];
+  Stage<BITS, GRP> st[Tr<BITS, GRP>::kS];
   float qs[kG * kD];                  // q of the pair's current segment, * scale * log2e / eps,
                                       // swizzled (qs_index)
   float part[2][kTB * 32];            // score partials, double-buffered (part_index)
-  float pv[kTB][20];                  // p' = p * s_v of token t, group g, head h at [t][4g + h];
-                                      // four entries pad the row
-  unsigned long long full[Tr<BITS>::kS];    // copies landed
-  unsigned long long empty[Tr<BITS>::kS];   // V-warp done with the stage
+  float pv[kTB][Tr<BITS, GRP>::kPvW];  // g32: p' = p * s_v of token t, group g, head h at
+                                      // [t][4g + h], four entries pad the row; g8: p of token
+                                      // t, head h at [t][h] (the V scale goes on the codes)
+  unsigned long long full[Tr<BITS, GRP>::kS];    // copies landed
+  unsigned long long empty[Tr<BITS, GRP>::kS];   // V-warp done with the stage
   unsigned long long pfull[2];        // S-warp wrote part[i]
   unsigned long long pempty[2];       // V-warp read part[i]
 };
 
-static_assert(sizeof(Stage<4>) % 16 == 0 && sizeof(Stage<8>) % 16 == 0, "stage alignment");
-static_assert(sizeof(PairSmem<4>) % 16 == 0 && sizeof(PairSmem<8>) % 16 == 0, "pair alignment");
+static_assert(sizeof(Stage<4, 32>) % 16 == 0 && sizeof(Stage<8, 32>) % 16 == 0 &&
+                  sizeof(Stage<4, 8>) % 16 == 0 && sizeof(Stage<8, 8>) % 16 == 0,
+              "stage alignment");
+static_assert(sizeof(PairSmem<4, 32>) % 16 == 0 && sizeof(PairSmem<8, 32>) % 16 == 0 &&
+                  sizeof(PairSmem<4, 8>) % 16 == 0 && sizeof(PairSmem<8, 8>) % 16 == 0,
+              "pair alignment");
 
 struct DecodeParams {
   const void* Q;
@@ -119,9 +130,9 @@ struct DecodeParams {
 };
 
 // shared memory after the pairs: pre [B + 1], len [B]
-template <int BITS>
+template <int BITS, int GRP>
 size_t smem_bytes(int B) {
-  return sizeof(PairSmem<BITS>) * Tr<BITS>::kNP + sizeof(int) * (2 * B + 1);
+  return sizeof(PairSmem<BITS, GRP>) * Tr<BITS, GRP>::kNP + sizeof(int) * (2 * B + 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -261,6 +272,15 @@ __device__ __forceinline__ int qs_index(int h, int c) {
   return h * kD + cs * 16 + ((j ^ ((cs >> 1) & 3)) << 2) + (c & 3);
 }
 
+// Token of lane group ts at iteration it of a block.  g32: tokens 4 it + ts,
+// all of one K group.  g8: lane group ts owns K group ts (tokens 8 ts ..
+// 8 ts + 7), visited in a rotated order so that the four groups' code rows
+// fall in both halves of the shared-memory banks.
+template <int GRP>
+__device__ __forceinline__ int block_token(int it, int ts) {
+  return GRP == 32 ? 4 * it + ts : 8 * ts + ((it + ts) & 7);
+}
+
 // Score partials of token t: the eight channel slices' float4 (one value per
 // head) in a 128-byte row, slice i at float4 (i ^ (t & 7)) so that eight
 // lanes reading slice i of eight tokens hit eight different bank groups.
@@ -323,34 +343,36 @@ __device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H
 
 // Lane 0 arms the stage's barrier with the block's byte count and issues the
 // four copies: K codes, V codes, the K scale row and the V scales.
-template <int BITS>
-__device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS>& ps, int stage, int b,
+template <int BITS, int GRP>
+__device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS, GRP>& ps, int stage, int b,
                                             int h, int j, const int* slen) {
   const long long head = static_cast<long long>(b) * p.H + h;
   const int len = slen[b];
   const int t0 = j * kTB;
   const int nv = min(kTB, len - t0);
-  constexpr int kCb = Tr<BITS>::kCb;
-  Stage<BITS>& st = ps.st[stage];
+  constexpr int kCb = Tr<BITS, GRP>::kCb;
+  Stage<BITS, GRP>& st = ps.st[stage];
   unsigned long long* bar = &ps.full[stage];
-  mbar_expect_tx(bar, static_cast<uint32_t>((2 * kCb + 16) * nv + 512));
+  constexpr int kVs = Tr<BITS, GRP>::kVs;
+  const int krows = (nv + GRP - 1) / GRP;                // K groups holding valid tokens
+  mbar_expect_tx(bar, static_cast<uint32_t>((2 * kCb + kVs * 4) * nv + krows * kD * 4));
   bulk_g2s(st.kc, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
   bulk_g2s(st.vc, p.v_codes + head * p.v_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
-  bulk_g2s(st.ks, p.k_scales + head * p.k_scales_head + static_cast<long long>(j) * kD,
-           kD * sizeof(float), bar);
-  bulk_g2s(st.vs, p.v_scales + head * p.v_scales_head + static_cast<long long>(t0) * (kD / 32),
-           nv * 16, bar);
+  bulk_g2s(st.ks, p.k_scales + head * p.k_scales_head + static_cast<long long>(t0 / GRP) * kD,
+           krows * kD * sizeof(float), bar);
+  bulk_g2s(st.vs, p.v_scales + head * p.v_scales_head + static_cast<long long>(t0) * kVs,
+           nv * kVs * 4, bar);
 }
 
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int BITS>
-__global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) decode_kernel(DecodeParams p) {
+template <int BITS, int GRP>
+__global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasPerSm) decode_kernel(DecodeParams p) {
   griddep_wait();
-  constexpr int kNP = Tr<BITS>::kNP, kS = Tr<BITS>::kS, kThreads = Tr<BITS>::kThreads;
-  using PairSmem = kvq::PairSmem<BITS>;
-  using Stage = kvq::Stage<BITS>;
+  constexpr int kNP = Tr<BITS, GRP>::kNP, kS = Tr<BITS, GRP>::kS, kThreads = Tr<BITS, GRP>::kThreads;
+  using PairSmem = kvq::PairSmem<BITS, GRP>;
+  using Stage = kvq::Stage<BITS, GRP>;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   PairSmem* pairs = reinterpret_cast<PairSmem*>(smem_raw);
   int* pre = reinterpret_cast<int*>(pairs + kNP);       // [B + 1]
@@ -403,7 +425,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
   // q * scale * log2e / eps into the pair's qs (the channel of value r is
   // lane + 32 r, so its parity is the lane's)
   auto store_q = [&]() {
-    const float qf = p.qscale * ((lane & 1) ? Tr<BITS>::kInvEpsOdd : Tr<BITS>::kInvEpsEven);
+    const float qf = p.qscale * ((lane & 1) ? Tr<BITS, GRP>::kInvEpsOdd : Tr<BITS, GRP>::kInvEpsEven);
 #pragma unroll
     for (int r = 0; r < kPer; ++r) {
       const int i = lane + 32 * r;
@@ -413,7 +435,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
   if (is_s) {
     load_q(seg);
     for (int s = 0; s < kS && prod.valid; ++s) {
-      if (lane == 0) issue_block<BITS>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
+      if (lane == 0) issue_block<BITS, GRP>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
       ++prod.j;
       prod = prod_settle(prod, pre, p.B, H, cr);
     }
@@ -447,11 +469,13 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
         u64 q2[kG][8];
         u64 kcp[kG];
         {
-          const ulonglong2* ksv = reinterpret_cast<const ulonglong2*>(st.ks + 16 * cs);
+          // the K scales of this lane's group: the block's one group (g32) or
+          // group ts (g8)
+          const ulonglong2* ksv = reinterpret_cast<const ulonglong2*>(st.ks[GRP == 32 ? 0 : ts] + 16 * cs);
           ulonglong2 kv2[4];
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) kv2[jj] = ksv[jj];
-          const u64 corr = pack2(Tr<BITS>::kCorrEven, Tr<BITS>::kCorrOdd);
+          const u64 corr = pack2(Tr<BITS, GRP>::kCorrEven, Tr<BITS, GRP>::kCorrOdd);
 #pragma unroll
           for (int hh = 0; hh < kG; ++hh) {
             u64 c2 = 0ull;
@@ -472,7 +496,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
         float* part = ps.part[pb];
 #pragma unroll 2
         for (int it = 0; it < kTB / 4; ++it) {
-          const int t = 4 * it + ts;
+          const int t = block_token<GRP>(it, ts);
           u64 f[8];
           code_pairs<BITS>(st.kc, t, cs, f);
           u64 acc[kG];
@@ -496,7 +520,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
           // the V-warp's reads of the stage happen before its arrive on
           // `empty`, which this wait acquires: the copy cannot overtake them
           wait_bar(&ps.empty[sp], (kp / kS) & 1u, p.err);
-          if (lane == 0) issue_block<BITS>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
+          if (lane == 0) issue_block<BITS, GRP>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
           ++prod.j;
           prod = prod_settle(prod, pre, p.B, H, cr);
         }
@@ -513,7 +537,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
         for (int i = 0; i < 8; ++i) u[hh][i] = 0ull;
       }
       const int g = cs >> 1;                            // V group of channels 16cs..16cs+15
-      const u64 ncorr = pack2(-Tr<BITS>::kCorrEven, -Tr<BITS>::kCorrOdd);
+      const u64 ncorr = pack2(-Tr<BITS, GRP>::kCorrEven, -Tr<BITS, GRP>::kCorrOdd);
       for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
@@ -558,8 +582,8 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
             for (int i = 0; i < 8; ++i) u[hh][i] = mul2(u[hh][i], a2);
           }
         }
-        // p' = p * s_v of this lane's token for each V group, as (p', p') pairs
-        {
+        if (GRP == 32) {
+          // p' = p * s_v of this lane's token for each V group, as (p', p') pairs
           const float4 sv = *reinterpret_cast<const float4*>(st.vs[lane]);
           const float svg[4] = {sv.x, sv.y, sv.z, sv.w};
           const u64 p01 = pack2(pr[0], pr[1]), p23 = pack2(pr[2], pr[3]);
@@ -570,14 +594,17 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
             *reinterpret_cast<ulonglong2*>(&ps.pv[lane][4 * gg]) =
                 make_ulonglong2(mul2(p01, s2), mul2(p23, s2));
           }
+        } else {
+          // g8: p itself; the V scales go on the codes
+          *reinterpret_cast<float4*>(&ps.pv[lane][0]) = make_float4(pr[0], pr[1], pr[2], pr[3]);
         }
         __syncwarp();
 
         // values: lane (ts, cs), token 4*it + ts, channels 16cs..16cs+15
 #pragma unroll 2
         for (int it = 0; it < kTB / 4; ++it) {
-          const int t = 4 * it + ts;
-          const float4 p4 = *reinterpret_cast<const float4*>(&ps.pv[t][4 * g]);
+          const int t = block_token<GRP>(it, ts);
+          const float4 p4 = *reinterpret_cast<const float4*>(&ps.pv[t][GRP == 32 ? 4 * g : 0]);
           u64 f[8];
           code_pairs<BITS>(st.vc, t, cs, f);
           const u64 pp[kG] = {pack2(p4.x, p4.x), pack2(p4.y, p4.y), pack2(p4.z, p4.z),
@@ -586,6 +613,19 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
           // contributes exactly zero
 #pragma unroll
           for (int i = 0; i < 8; ++i) f[i] = add2(f[i], ncorr);
+          if (GRP == 8) {
+            // the scales of V groups 2 cs and 2 cs + 1 (channels 16 cs .. +7,
+            // +8 .. +15); zero past the length, where the stage holds stale
+            // scales and p is already zero
+            const float2 sv = *reinterpret_cast<const float2*>(&st.vs[t][2 * cs]);
+            const bool tv = t < nvalid;
+            const u64 s0 = pack2(tv ? sv.x : 0.f, tv ? sv.x : 0.f), s1 = pack2(tv ? sv.y : 0.f, tv ? sv.y : 0.f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              f[i] = mul2(f[i], s0);
+              f[4 + i] = mul2(f[4 + i], s1);
+            }
+          }
 #pragma unroll
           for (int hh = 0; hh < kG; ++hh)
 #pragma unroll
@@ -610,7 +650,7 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           // u carries a factor eps of the channel: scale it back
-          float x = lo_f(u[hh][i]) * Tr<BITS>::kInvEpsEven, y = hi_f(u[hh][i]) * Tr<BITS>::kInvEpsOdd;
+          float x = lo_f(u[hh][i]) * Tr<BITS, GRP>::kInvEpsEven, y = hi_f(u[hh][i]) * Tr<BITS, GRP>::kInvEpsOdd;
           x += __shfl_xor_sync(0xffffffffu, x, 8);
           y += __shfl_xor_sync(0xffffffffu, y, 8);
           x += __shfl_xor_sync(0xffffffffu, x, 16);
@@ -650,16 +690,36 @@ __global__ void __launch_bounds__(Tr<BITS>::kThreads, Tr<BITS>::kCtasPerSm) deco
 // per SM, 1 KB of it reserved per CTA, at most 227 KB per CTA).
 constexpr size_t smem_limit(int per_sm) { return per_sm == 1 ? 227 * 1024 : 113 * 1024; }
 
+// The instantiation for a call's code width and group size: its launch shape
+// and kernel.
+struct DecodeVariant {
+  int pairs, per_sm, threads;
+  size_t (*smem)(int B);
+  void (*kernel)(DecodeParams);
+};
+
+template <int BITS, int GRP>
+DecodeVariant variant_of() {
+  return {Tr<BITS, GRP>::kNP, Tr<BITS, GRP>::kCtasPerSm, Tr<BITS, GRP>::kThreads, smem_bytes<BITS, GRP>,
+          decode_kernel<BITS, GRP>};
+}
+
+DecodeVariant variant(const AttendArgs& a) {
+  if (a.g.group == 32) return a.g.bits == 4 ? variant_of<4, 32>() : variant_of<8, 32>();
+  return a.g.bits == 4 ? variant_of<4, 8>() : variant_of<8, 8>();
+}
+
 bool decode_applies(const AttendArgs& a) {
-  return (a.g.bits == 4 || a.g.bits == 8) && a.g.group == kTB && a.g.D == kD && a.Lq == 1 &&
-         a.H_q == kG * a.g.H_kv &&
-         (a.g.bits == 4 ? smem_bytes<4>(a.g.B) <= smem_limit(Tr<4>::kCtasPerSm)
-                        : smem_bytes<8>(a.g.B) <= smem_limit(Tr<8>::kCtasPerSm));
+  if (!((a.g.bits == 4 || a.g.bits == 8) && (a.g.group == 32 || a.g.group == 8) && a.g.D == kD &&
+        a.Lq == 1 && a.H_q == kG * a.g.H_kv))
+    return false;
+  const DecodeVariant v = variant(a);
+  return v.smem(a.g.B) <= smem_limit(v.per_sm);
 }
 
 int decode_ctas(const AttendArgs& a) {
   const long long t_max = static_cast<long long>(a.g.B) * a.g.H_kv * ((a.g.N_cap + kTB - 1) / kTB);
-  const int per_sm = a.g.bits == 4 ? Tr<4>::kCtasPerSm : Tr<8>::kCtasPerSm;
+  const int per_sm = variant(a).per_sm;
   long long ctas = a.splits > 0 ? a.splits : static_cast<long long>(per_sm) * (sm_count() > 0 ? sm_count() : 148);
   if (ctas > t_max) ctas = t_max;
   if (ctas < 1) ctas = 1;
@@ -667,7 +727,7 @@ int decode_ctas(const AttendArgs& a) {
 }
 
 // Warp pairs per CTA: each pair is one worker of the plan.
-int decode_pairs(const AttendArgs& a) { return a.g.bits == 4 ? Tr<4>::kNP : Tr<8>::kNP; }
+int decode_pairs(const AttendArgs& a) { return variant(a).pairs; }
 
 size_t decode_workspace(const AttendArgs& a) {
   return with_window_slots(a, partial_slots(decode_ctas(a) * decode_pairs(a), a.g.B, a.g.H_kv),
@@ -676,10 +736,10 @@ size_t decode_workspace(const AttendArgs& a) {
 
 kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   const int ctas = decode_ctas(a);
-  const bool b4 = a.g.bits == 4;
-  const size_t smem = b4 ? smem_bytes<4>(a.g.B) : smem_bytes<8>(a.g.B);
-  auto kernel = b4 ? decode_kernel<4> : decode_kernel<8>;
-  const int threads = b4 ? Tr<4>::kThreads : Tr<8>::kThreads;
+  const DecodeVariant v = variant(a);
+  const size_t smem = v.smem(a.g.B);
+  auto kernel = v.kernel;
+  const int threads = v.threads;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return KVQ_ERR_CUDA;
@@ -730,7 +790,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   return launch_merge(m, s);
 }
 
-const AttendImpl kDecode{"decode_gqa4_d128_g32", decode_applies, decode_workspace, decode_launch};
+const AttendImpl kDecode{"decode_gqa4_d128", decode_applies, decode_workspace, decode_launch};
 
 }  // namespace
 

@@ -24,6 +24,7 @@ namespace {
 constexpr int kWT = 32;          // window tokens per tile
 constexpr int kWR = 32;          // rows per pass
 constexpr int kWThreads = 256;
+static_assert(kWT == 32, "the softmax of a tile runs one token per lane");
 
 struct WindowParams {
   WindowArgs a;
@@ -59,10 +60,20 @@ __global__ void __launch_bounds__(kWThreads) window_kernel(WindowParams wp) {
   const long long win_base = static_cast<long long>(bh) * a.W_cap * D;
   float* slot = a.partials + (a.slot0 + bh) * a.slot_stride;
 
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int r0 = 0; r0 < R; r0 += kWR) {
     const int rows = min(kWR, R - r0);
-    for (int i = threadIdx.x; i < rows * D; i += blockDim.x)
-      s_q[i] = load_as_f32(a.Q, (row_base + r0) * D + i, a.q_dtype);
+    for (int i0 = threadIdx.x; i0 < rows * D; i0 += kWThreads * 8) {
+      float qv[8];                                     // eight loads in flight per thread
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kWThreads;
+        qv[u] = i < rows * D ? load_as_f32(a.Q, (row_base + r0) * D + i, a.q_dtype) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (i0 + u * kWThreads < rows * D) s_q[i0 + u * kWThreads] = qv[u];
+    }
     for (int i = threadIdx.x; i < kWR * D; i += blockDim.x) s_u[i] = 0.f;
     if (threadIdx.x < kWR) {
       s_m[threadIdx.x] = -INFINITY;
@@ -71,11 +82,26 @@ __global__ void __launch_bounds__(kWThreads) window_kernel(WindowParams wp) {
     __syncthreads();
     for (int t0 = 0; t0 < wl; t0 += kWT) {
       const int nt = min(kWT, wl - t0);
-      for (int i = threadIdx.x; i < kWT * D; i += blockDim.x) {
-        const int t = i / D, d = i - t * D;
-        const bool live = t < nt;
-        s_k[t * DS + d] = live ? load_as_f32(a.K_win, win_base + static_cast<long long>(t0 + t) * D + d, a.win_dtype) : 0.f;
-        s_v[t * DS + d] = live ? load_as_f32(a.V_win, win_base + static_cast<long long>(t0 + t) * D + d, a.win_dtype) : 0.f;
+      // the tile's K and V rows, all of a thread's loads issued before any store
+      for (int i0 = threadIdx.x; i0 < kWT * D; i0 += kWThreads * 8) {
+        float kv[8], vv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kWThreads;
+          const bool live = i < nt * D;
+          const long long e = win_base + static_cast<long long>(t0) * D + i;
+          kv[u] = live ? load_as_f32(a.K_win, e, a.win_dtype) : 0.f;
+          vv[u] = live ? load_as_f32(a.V_win, e, a.win_dtype) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kWThreads;
+          if (i < kWT * D) {
+            const int t = i / D, d = i - t * D;
+            s_k[t * DS + d] = kv[u];
+            s_v[t * DS + d] = vv[u];
+          }
+        }
       }
       __syncthreads();
       // scores of the tile
@@ -90,23 +116,27 @@ __global__ void __launch_bounds__(kWThreads) window_kernel(WindowParams wp) {
         s_p[i] = sc;
       }
       __syncthreads();
-      // the block rule: m_new = max(m, tile max), alpha = exp(m - m_new)
-      if (threadIdx.x < rows) {
-        const int r = threadIdx.x;
-        float mb = -INFINITY;
-        for (int t = 0; t < nt; ++t) mb = fmaxf(mb, s_p[r * kWT + t]);
+      // the block rule: m_new = max(m, tile max), alpha = exp(m - m_new);
+      // a warp per row, lane = token of the tile
+      for (int r = warp; r < rows; r += kWThreads / 32) {
+        const float sc = s_p[r * kWT + lane];          // -inf past the tile's tokens
+        float mb = sc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
         const float mo = s_m[r];
         const float mn = fmaxf(mo, mb);
-        const float al = mo == -INFINITY ? 0.f : expf(mo - mn);
-        float zs = 0.f;
-        for (int t = 0; t < kWT; ++t) {
-          const float e = t < nt ? expf(s_p[r * kWT + t] - mn) : 0.f;
-          s_p[r * kWT + t] = e;
-          zs += e;
+        const float e = lane < nt ? expf(sc - mn) : 0.f;
+        float zs = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+        s_p[r * kWT + lane] = e;
+        __syncwarp();
+        if (lane == 0) {
+          const float al = mo == -INFINITY ? 0.f : expf(mo - mn);
+          s_z[r] = al * s_z[r] + zs;
+          s_m[r] = mn;
+          s_a[r] = al;
         }
-        s_z[r] = al * s_z[r] + zs;
-        s_m[r] = mn;
-        s_a[r] = al;
       }
       __syncthreads();
       for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {

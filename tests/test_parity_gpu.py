@@ -451,3 +451,30 @@ def test_window_bad_lengths(sm):
     with pytest.raises(sm.KVQError):
         sm.check()
     sm.check()
+
+
+# ---------------------------------------------------------------------------
+# tuned decode at group size 8
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_decode_g8(sm, bits):
+    """The tuned decode kernel at g = 8 (four K scale rows per 32-token block,
+    sixteen V scales per token): lengths ending inside a K group of 8 and
+    inside a block, one shorter than a group, outlier channels, splits."""
+    q, k, v, lens = _gqa_case(4, 8, 2, 700, 128, [700, 301, 128, 5], seed=70 + bits, bits=bits, outliers=True)
+    cache = pack_gpu(sm, k, v, bits, 8)
+    assert sm.kernel_name(cache, 8, 1).startswith("decode_gqa4")
+    for splits in (0, 1, 5):
+        _check_gqa(sm, q, k, v, lens, bits, 8, 1.0, splits=splits)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_decode_g8_zero_and_window(sm, bits):
+    """g = 8: a zero V cache gives exact zeros; and a window on top."""
+    q, k, v, lens = _gqa_case(2, 8, 2, 300, 128, [300, 157], seed=72 + bits)
+    v0 = np.zeros_like(v)
+    o = _check_gqa(sm, q, k, v0, lens, bits, 8, 1.0)
+    assert np.all(o == 0.0)
+    kw, vw, wl = _window(2, 2, 16, 128, [9, 16], seed=73)
+    _check_window(sm, q, k, v, lens, kw, vw, wl, bits, 8, 1.0)
