@@ -130,6 +130,11 @@ class PackedCache:
         self.v_codes = torch.zeros(vc, dtype=torch.uint8, device=dev)
         self.v_scales = torch.zeros(vs // 4, dtype=torch.float32, device=dev)
         self.device = dev
+        # the four buffers never move, so the C struct is built once
+        self._struct = _Cache(self.bits, self.group, self.B, self.H_kv, self.N_cap, self.D,
+                              self.k_codes.data_ptr(), self.k_scales.data_ptr(),
+                              self.v_codes.data_ptr(), self.v_scales.data_ptr())
+        self._ws = {}                      # (H_q, Lq, splits, window) -> workspace bytes
 
     @property
     def Np(self) -> int:
@@ -144,9 +149,16 @@ class PackedCache:
                    (self.k_codes, self.k_scales, self.v_codes, self.v_scales))
 
     def struct(self) -> _Cache:
-        return _Cache(self.bits, self.group, self.B, self.H_kv, self.N_cap, self.D,
-                      self.k_codes.data_ptr(), self.k_scales.data_ptr(),
-                      self.v_codes.data_ptr(), self.v_scales.data_ptr())
+        return self._struct
+
+    def _workspace_bytes(self, H_q: int, Lq: int, splits: int, window: bool) -> int:
+        key = (H_q, Lq, splits, window)
+        n = self._ws.get(key)
+        if n is None:
+            f = lib.kvq_workspace_size_window if window else lib.kvq_workspace_size
+            n = int(f(ctypes.byref(self._struct), int(H_q), int(Lq), int(splits)))
+            self._ws[key] = n
+        return n
 
     # per-(b, h) views, for tests and inspection
     def head_k_codes(self, b: int, h: int) -> torch.Tensor:
@@ -195,8 +207,7 @@ def pack(K: torch.Tensor | None, V: torch.Tensor | None, cache: PackedCache, t0:
 
 
 def workspace_size(cache: PackedCache, H_q: int, Lq: int, splits: int = 0) -> int:
-    c = cache.struct()
-    return int(lib.kvq_workspace_size(ctypes.byref(c), int(H_q), int(Lq), int(splits)))
+    return cache._workspace_bytes(int(H_q), int(Lq), int(splits), False)
 
 
 def kernel_name(cache: PackedCache, H_q: int, Lq: int) -> str:
@@ -258,8 +269,7 @@ def attend_noalloc(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, s
 
 
 def workspace_size_window(cache: PackedCache, H_q: int, Lq: int, splits: int = 0) -> int:
-    c = cache.struct()
-    return int(lib.kvq_workspace_size_window(ctypes.byref(c), int(H_q), int(Lq), int(splits)))
+    return cache._workspace_bytes(int(H_q), int(Lq), int(splits), True)
 
 
 def attend_window(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, K_win: torch.Tensor,

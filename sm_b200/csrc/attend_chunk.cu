@@ -707,9 +707,7 @@ bool make_q_map(const AttendArgs& a, CUtensorMap* map) {
 kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   const int ctas = chunk_ctas(a);
   const size_t smem = smem_bytes(a.g.B);
-  if (cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return KVQ_ERR_CUDA;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(chunk_kernel), smem)) return KVQ_ERR_CUDA;
   CUtensorMap qmap;
   if (!make_q_map(a, &qmap)) return KVQ_ERR_CUDA;
   ChunkParams p{};

@@ -740,9 +740,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   const size_t smem = v.smem(a.g.B);
   auto kernel = v.kernel;
   const int threads = v.threads;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
-    return KVQ_ERR_CUDA;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kernel), smem)) return KVQ_ERR_CUDA;
   DecodeParams p{};
   p.Q = a.Q;
   p.q_dtype = a.q_dtype;

@@ -217,9 +217,7 @@ kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
   const size_t smem = smem_bytes(a.g.D, a.g.B);
   if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
   if (n_rt > 65535) return KVQ_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(attend_generic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return KVQ_ERR_CUDA;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(attend_generic_kernel), smem)) return KVQ_ERR_CUDA;
   GenericParams p{};
   p.Q = a.Q;
   p.q_dtype = a.q_dtype;

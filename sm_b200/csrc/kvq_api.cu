@@ -43,6 +43,28 @@ int sm_count() {
   return cache[dev];
 }
 
+bool ensure_dynamic_smem(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<int, const void*>, size_t>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& e : done)
+    if (e.first.first == dev && e.first.second == kernel) {
+      if (e.second >= bytes) return true;
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+          cudaSuccess)
+        return false;
+      e.second = bytes;
+      return true;
+    }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess)
+    return false;
+  done.push_back({{dev, kernel}, bytes});
+  return true;
+}
+
 bool make_geometry(const kvq_cache* c, Geometry* g) {
   if (!c) return false;
   if (c->bits != 4 && c->bits != 8) return false;

@@ -28,6 +28,11 @@ void count_launch(int n = 1);
 // SM count of the current device (cached per device)
 int sm_count();
 
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes) on the
+// current device unless an equal or larger value was already set there:
+// the attribute call costs host time on every launch otherwise.
+bool ensure_dynamic_smem(const void* kernel, size_t bytes);
+
 // ---------------------------------------------------------------------------
 // cache geometry
 // ---------------------------------------------------------------------------

@@ -215,9 +215,7 @@ kvq_status launch_pack(const PackArgs& a, cudaStream_t s) {
     const size_t smem = (static_cast<size_t>(g.group) * g.D + 2 * g.D) * sizeof(float);
     if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
     if (smem > 48 * 1024) {
-      if (cudaFuncSetAttribute(pack_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return KVQ_ERR_CUDA;
+      if (!ensure_dynamic_smem(reinterpret_cast<const void*>(pack_k_kernel), smem)) return KVQ_ERR_CUDA;
     }
     PackParams pk{a.K, a.in_dtype, a.t0, T, g.bits, g.group, g.B, g.H_kv, g.D, g.Dp,
                   static_cast<long long>(g.k_codes_head), static_cast<long long>(g.k_scales_head),

@@ -193,9 +193,7 @@ kvq_status launch_window(const WindowArgs& w, cudaStream_t s) {
   const long long blocks = static_cast<long long>(w.B) * w.H_kv;
   if (blocks > 0x7fffffffLL || w.D > 256 || w.D < 1) return KVQ_ERR_UNSUPPORTED;
   const size_t smem = window_smem(w.D);
-  if (cudaFuncSetAttribute(window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
-    return KVQ_ERR_CUDA;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(window_kernel), smem)) return KVQ_ERR_CUDA;
   WindowParams p{w};
   if (launch_pdl(window_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kWThreads), smem, s, p) != cudaSuccess)
     return KVQ_ERR_CUDA;
