@@ -144,6 +144,23 @@ KVQ_API kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache*
                       void* workspace, size_t ws_bytes, int32_t splits, void* stream);
 
 /*
+ * Causal multi-query attention over the packed cache (chunked prefill): the
+ * Lq query rows of sequence b are its last Lq positions, L - Lq .. L - 1
+ * (L = lengths[b], the tokens already packed), and query i reads keys
+ * [0, L - Lq + i] only; keys after a query's position take no part in its
+ * max or sum ("给长前缀列一张有单位的资源账本", section
+ * "FlashAttention为什么不必保存整张热图").  The pages' own studies are
+ * non-causal; this is the masked form of the same rule.  Arguments, layout,
+ * workspace (kvq_workspace_size) and errors as kvq_attend; a sequence with
+ * L < Lq is also reported (KVQ_ERR_LENGTH) and its rows without a visible
+ * key are zeros.  With Lq = 1 it is kvq_attend.
+ */
+KVQ_API kvq_status kvq_attend_causal(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                     const int32_t* lengths, int32_t H_q, int32_t Lq, float scale,
+                                     void* O, void* workspace, size_t ws_bytes, int32_t splits,
+                                     void* stream);
+
+/*
  * Attention of Q over the packed cache followed by a window of recent tokens
  * kept unquantized.  The pages leave this as their next study: keep the same
  * packed format and spend a limited high-precision budget on the most recent

@@ -50,6 +50,7 @@ from .kvq_oracle import (  # noqa: F401
     attend_gqa,
     attend_gqa_heads,
     attend_gqa_window,
+    attend_gqa_causal,
     rel_l2_error,
     pack_cache,
 )

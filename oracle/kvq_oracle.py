@@ -461,6 +461,37 @@ def attend_gqa_window(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, lengt
     return out
 
 
+def attend_gqa_causal(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray,
+                      lengths, scale: float) -> np.ndarray:
+    """Causal multi-query attention over decoded caches: the Lq query rows of
+    sequence b are its last Lq positions, L - Lq .. L - 1 (L = lengths[b]),
+    and query i reads keys [0, L - Lq + i] only.  Keys after a query's own
+    position are masked: they enter neither the max nor the sum
+    ("给长前缀列一张有单位的资源账本", section "FlashAttention为什么不必保存整张
+    热图").  The pages' own studies are non-causal ("注意力分塊", opening
+    section, which names causal training prefill as something its method
+    does not replace); this is the masked form their rule gives.  GQA as in
+    ``attend_gqa``.  Returns float64 [B, H_q, Lq, D]; a row with no visible
+    key (L < Lq) raises.
+    """
+    b_, hq, lq, d = q.shape
+    hkv = k_hat.shape[1]
+    if hq % hkv:
+        raise ValueError("H_q must be a multiple of H_kv")
+    grp = hq // hkv
+    out = np.zeros((b_, hq, lq, v_hat.shape[-1]), np.float64)
+    for b in range(b_):
+        n = int(lengths[b])
+        for h in range(hq):
+            for i in range(lq):
+                visible = n - lq + i + 1
+                if visible <= 0:
+                    raise ValueError("a row with no valid key has no softmax")
+                out[b, h, i] = attend_dense(q[b, h, i:i + 1], k_hat[b, h // grp, :visible],
+                                            v_hat[b, h // grp, :visible], scale)[0]
+    return out
+
+
 def rel_l2_error(out: np.ndarray, ref: np.ndarray) -> float:
     """||out - ref||_2 / ||ref||_2 over the whole output ("KV分组打包", section
     "同一输入上的精度与空间交换": relative L2 output error per input, then the

@@ -78,6 +78,9 @@ def _load() -> ctypes.CDLL:
     L.kvq_attend_noalloc.restype = ctypes.c_int
     L.kvq_noalloc_scratch_bytes.argtypes = []
     L.kvq_noalloc_scratch_bytes.restype = sz
+    L.kvq_attend_causal.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, i32, i32,
+                                    ctypes.c_float, vp, vp, sz, i32, vp]
+    L.kvq_attend_causal.restype = ctypes.c_int
     L.kvq_attend_window.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, vp, vp, ctypes.c_int,
                                     vp, i32, i32, i32, ctypes.c_float, vp, vp, sz, i32, vp]
     L.kvq_attend_window.restype = ctypes.c_int
@@ -217,10 +220,11 @@ def kernel_name(cache: PackedCache, H_q: int, Lq: int) -> str:
 
 def attend(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, scale: float,
            out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-           splits: int = 0) -> torch.Tensor:
+           splits: int = 0, causal: bool = False) -> torch.Tensor:
     """O = softmax(scale * Q K^T) V over the packed cache, per sequence up to
     its length.  Q [B, H_q, Lq, D] fp32/bf16; lengths int32 [B] on the device;
-    returns O like Q (written into ``out`` if given)."""
+    returns O like Q (written into ``out`` if given).  causal: the Lq rows are
+    the sequence's last Lq positions and row i reads keys [0, L - Lq + i]."""
     _check_cuda(Q, "Q", cache.device)
     _check_cuda(lengths, "lengths", cache.device)
     if lengths.dtype != torch.int32 or lengths.numel() != cache.B:
@@ -238,10 +242,11 @@ def attend(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, scale: fl
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=cache.device)
     c = cache.struct()
-    _ok(lib.kvq_attend(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(), H_q, Lq,
-                       float(scale), out.data_ptr(), workspace.data_ptr(),
-                       workspace.numel() * workspace.element_size(), int(splits),
-                       _stream(cache.device)), "kvq_attend")
+    fn = lib.kvq_attend_causal if causal else lib.kvq_attend
+    _ok(fn(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(), H_q, Lq,
+           float(scale), out.data_ptr(), workspace.data_ptr(),
+           workspace.numel() * workspace.element_size(), int(splits),
+           _stream(cache.device)), "kvq_attend_causal" if causal else "kvq_attend")
     return out
 
 

@@ -107,6 +107,7 @@ struct ChunkParams {
   float* partials;                       // [slots][kD + 2][R]: m, z, u (feature-major)
   int ctas;
   int force_partial;                     // a window follows: no CTA writes output rows
+  int causal;                            // query i of Lq reads keys [0, len - Lq + i] only
   unsigned int* err;
 };
 
@@ -526,6 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
       const uint32_t o_col = tmem + lane_addr + 256u + 128u * tile;
       const bool neg = p.qscale < 0.f;
       const float aq = fabsf(p.qscale);
+      // the row's query index within its head (rows are head-major, Lq each)
+      const int qi = (128 * tile + r) % p.Lq;
       if (tile < p.NT) {
         float m_ref = -INFINITY, z = 0.f;
         Cursor c;
@@ -537,7 +540,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
           }
           wait_bar(bar(S_FULL + tile), k & 1u, p.err, abort_flag);
           tc_fence_after();
-          const int nv = min(kBT, slen[c.seg.b] - c.j * kBT);
+          // valid columns of this row: the sequence end, and with a causal
+          // mask the row's own position (none at all if this block starts
+          // after it; m_ref then stays -inf and every p is zero)
+          const int nv_seq = min(kBT, slen[c.seg.b] - c.j * kBT);
+          const int nv = p.causal ? min(nv_seq, slen[c.seg.b] - p.Lq + qi + 1 - c.j * kBT) : nv_seq;
           // pass 1: the row's extreme over the valid columns, 64 at a time
           float mx = neg ? INFINITY : -INFINITY;
 #pragma unroll
@@ -613,7 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
               part[0] = m_ref * kLn2;
               part[p.R] = z;
             }
-            const float inv = 1.f / z;
+            // z = 0: a causal row with no visible key (length < Lq, reported by the merge)
+            const float inv = z > 0.f ? 1.f / z : 0.f;
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
               uint32_t orr[32];
@@ -733,6 +741,7 @@ kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   p.partials = static_cast<float*>(a.workspace);
   p.ctas = ctas;
   p.force_partial = a.win_lengths != nullptr;
+  p.causal = a.causal;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
   if (launch_pdl(chunk_kernel, dim3(ctas), dim3(kThreads), smem, s, qmap, p) != cudaSuccess) return KVQ_ERR_CUDA;
@@ -753,6 +762,7 @@ kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   m.D = kD;
   m.G = p.G;
   m.Lq = a.Lq;
+  m.causal = a.causal;
   m.feature_major = true;
   const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(ctas, a.g.B, a.g.H_kv)),
                                    static_cast<long long>(kD + 2) * p.R, 1, p.R, &m, s);

@@ -35,6 +35,7 @@ struct GenericParams {
   float* partials;             // [slots][n_rt*kRT][D + 2]
   int ctas;
   int force_partial;           // a window follows: no CTA writes output rows
+  int causal;                  // query i of Lq reads keys [0, len - Lq + i] only
 };
 
 __device__ __forceinline__ int code_at(const uint8_t* codes, long long flat, int bits) {
@@ -125,7 +126,9 @@ __global__ void __launch_bounds__(kThreads) attend_generic_kernel(GenericParams 
       for (int idx = threadIdx.x; idx < kRT * kBT; idx += blockDim.x) {
         const int r = idx / kBT, t = idx - r * kBT;
         float sc = -INFINITY;
-        if (r < rows && t < nt) {
+        // causal: key t_base + t is visible to query (r0 + r) % Lq up to its position
+        const bool seen = !p.causal || t_base + t <= len - p.Lq + (r0 + r) % p.Lq;
+        if (r < rows && t < nt && seen) {
           float acc = 0.f;
           for (int d = 0; d < D; ++d) acc = fmaf(s_q[r * D + d], s_k[t * DS + d], acc);
           sc = acc * p.scale;
@@ -142,7 +145,9 @@ __global__ void __launch_bounds__(kThreads) attend_generic_kernel(GenericParams 
         const float a = (mo == -INFINITY) ? 0.f : expf(mo - mn);
         float zs = 0.f;
         for (int t = 0; t < kBT; ++t) {
-          const float e = t < nt ? expf(s_p[r * kBT + t] - mn) : 0.f;
+          // a masked key is -inf, and so is mn while a causal row has seen no key
+          const float sc = s_p[r * kBT + t];
+          const float e = (t < nt && sc != -INFINITY) ? expf(sc - mn) : 0.f;
           s_p[r * kBT + t] = e;
           zs += e;
         }
@@ -163,7 +168,8 @@ __global__ void __launch_bounds__(kThreads) attend_generic_kernel(GenericParams 
     if (whole) {
       for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
         const int r = idx / D;
-        store_from_f32(p.O, row_base * D + idx, s_u[idx] / s_z[r], p.q_dtype);
+        // z = 0: a causal row with no visible key (length < Lq, reported by the merge)
+        store_from_f32(p.O, row_base * D + idx, s_z[r] > 0.f ? s_u[idx] / s_z[r] : 0.f, p.q_dtype);
       }
     } else {
       const long long slot = static_cast<long long>(blockIdx.x) + head;
@@ -246,6 +252,7 @@ kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
   p.partials = static_cast<float*>(a.workspace);
   p.ctas = ctas;
   p.force_partial = a.win_lengths != nullptr;
+  p.causal = a.causal;
   const cudaError_t le = launch_pdl(attend_generic_kernel, dim3(ctas, n_rt), dim3(kThreads), smem, s, p);
   if (le != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
@@ -265,6 +272,7 @@ kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
   m.D = a.g.D;
   m.G = p.G;
   m.Lq = a.Lq;
+  m.causal = a.causal;
   const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(ctas, a.g.B, a.g.H_kv)),
                                    static_cast<long long>(n_rt) * kRT * (a.g.D + 2), a.g.D + 2, 1, &m, s);
   if (ws != KVQ_OK) return ws;

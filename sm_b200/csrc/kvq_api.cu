@@ -182,13 +182,14 @@ size_t kvq_workspace_size(const kvq_cache* cache, int32_t H_q, int32_t Lq, int32
   return impl.workspace(a);
 }
 
-kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
-                      const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
-                      void* workspace, size_t ws_bytes, int32_t splits, void* stream) {
+static kvq_status attend_common(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
+                                void* workspace, size_t ws_bytes, int32_t splits, bool causal, void* stream) {
   AttendArgs a{};
   if (!fill_attend_args(Q, q_dtype, cache, lengths, H_q, Lq, scale, O, workspace, ws_bytes,
                         splits, &a))
     return KVQ_ERR_ARG;
+  a.causal = causal && Lq > 1;             // one query row at the last position sees every key
   if (!Q || !O || !lengths || !cache->k_codes || !cache->k_scales || !cache->v_codes ||
       !cache->v_scales)
     return KVQ_ERR_ARG;
@@ -207,6 +208,20 @@ kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
     if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
   }
   return impl.launch(a, static_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                      const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
+                      void* workspace, size_t ws_bytes, int32_t splits, void* stream) {
+  return attend_common(Q, q_dtype, cache, lengths, H_q, Lq, scale, O, workspace, ws_bytes, splits, false,
+                       stream);
+}
+
+kvq_status kvq_attend_causal(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                             const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
+                             void* workspace, size_t ws_bytes, int32_t splits, void* stream) {
+  return attend_common(Q, q_dtype, cache, lengths, H_q, Lq, scale, O, workspace, ws_bytes, splits, true,
+                       stream);
 }
 
 static bool fill_window(const void* K_win, const void* V_win, kvq_dtype win_dtype,

@@ -119,6 +119,7 @@ struct MergeArgs {
   int R, R_pad, D;                 // rows per (b,h) and the padded row count of a slot
   int G, Lq;                       // query heads per KV head, rows per query head
   bool feature_major;              // partial layout (rows contiguous per field)
+  bool causal;                     // causal rows: a length below Lq leaves rows without keys
   // recent-token window (kvq_attend_window); win_lengths == nullptr: none.
   // With a window every (b, h) is merged: its window state sits in slot
   // win_slot0 + b * H_kv + h, and no worker wrote an output row itself.
@@ -186,6 +187,7 @@ struct AttendArgs {
   void* workspace;
   size_t ws_bytes;
   int splits;
+  bool causal;                     // kvq_attend_causal: query i of Lq reads keys [0, len - Lq + i]
   // recent-token window (kvq_attend_window); win_lengths == nullptr: none
   const void* K_win;
   const void* V_win;

@@ -51,7 +51,7 @@ __device__ __forceinline__ MergePlan merge_plan(const MergeArgs& a, const int* s
     wl = wr < 0 ? 0 : (wr > a.W_cap ? a.W_cap : wr);
     bad = raw < 0 || raw > a.N_cap || wr < 0 || wr > a.W_cap || (nb == 0 && wl == 0);
   } else {
-    bad = raw < 1 || raw > a.N_cap;
+    bad = raw < 1 || raw > a.N_cap || (a.causal && raw < a.Lq);
   }
   if (report && bad) record_error(err, KVQ_ERR_LENGTH);
   MergePlan p{};
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams mp) {
           u = fmaf(w, uc, u);
         }
       }
-      store_from_f32(a.O, (row_base + r) * D + d, u / z, a.o_dtype);
+      store_from_f32(a.O, (row_base + r) * D + d, z > 0.f ? u / z : 0.f, a.o_dtype);
     }
     __syncthreads();
   }
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kMW * 32) merge_parts_kernel(MergeParams mp) {
       zt += s_z[w];
       ut += s_u[w][lane];
     }
-    store_from_f32(a.O, row * D + d, ut / zt, a.o_dtype);
+    store_from_f32(a.O, row * D + d, zt > 0.f ? ut / zt : 0.f, a.o_dtype);
   }
 }
 
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kFmThreads, 4) merge_fm_kernel(MergeParams mp)
 #pragma unroll
       for (int j = 0; j < 8; ++j) u[j] = fmaf(wgt[k], v[k][j], u[j]);
   }
-  const float inv = 1.f / z;
+  const float inv = z > 0.f ? 1.f / z : 0.f;      // z = 0: a causal row with no visible key
   if (a.o_dtype == KVQ_BF16 && nf == 8) {
     uint32_t o[4];
 #pragma unroll

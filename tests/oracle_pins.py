@@ -359,6 +359,34 @@ def pin_window():
                          - O.attend_gqa(q, k, v, [7, 4, 3], 0.7))) < 1e-12
 
 
+def pin_causal():
+    """Causal rows: brute force over each query's visible keys [0, L - Lq + i]
+    (keys past it filled with huge values so that reading them would show);
+    one query row is the plain cache; the last row of a chunk sees every
+    key, the first row L - Lq + 1 of them."""
+    rng = np.random.default_rng(23)
+    b_, hq, hkv, lq, n, d = 2, 4, 2, 3, 9, 5
+    q = rng.standard_normal((b_, hq, lq, d))
+    k = rng.standard_normal((b_, hkv, n, d))
+    v = rng.standard_normal((b_, hkv, n, d))
+    lens = [9, 5]
+    k[1, :, 5:] = 1e6
+    v[1, :, 5:] = -1e6
+    out = O.attend_gqa_causal(q, k, v, lens, 0.8)
+    for b in range(b_):
+        for h in range(hq):
+            hk = h // (hq // hkv)
+            for i in range(lq):
+                vis = lens[b] - lq + i + 1
+                bf = O.attend_bruteforce(q[b, h, i:i + 1], k[b, hk, :vis], v[b, hk, :vis], 0.8)
+                assert np.max(np.abs(out[b, h, i] - bf[0])) < 1e-12
+    full = O.attend_gqa(q, k, v, lens, 0.8)
+    assert np.max(np.abs(out[:, :, -1] - full[:, :, -1])) < 1e-12
+    assert np.max(np.abs(out[:, :, 0] - full[:, :, 0])) > 1e-3      # the first row sees fewer keys
+    one = O.attend_gqa_causal(q[:, :, :1], k, v, lens, 0.8)
+    assert np.max(np.abs(one - O.attend_gqa(q[:, :, :1], k, v, lens, 0.8))) < 1e-12
+
+
 def pin_rel_l2_band():
     """Soft check (parity unpinned at the value level): the mean relative L2
     output error on the six clean inputs lands near the pages' table, and the
@@ -387,4 +415,5 @@ ALL_PINS = [
     pin_eight_bit, pin_ledger, pin_workspace_sizes, pin_17_over_3,
     pin_negative_example, pin_dense_vs_blocked, pin_bruteforce,
     pin_large_scores_stay_finite, pin_merge_partials, pin_gqa_and_lengths, pin_window,
+    pin_causal,
 ]

@@ -167,6 +167,18 @@ def _window_before_packed_length(q, k_hat, v_hat, lengths, k_win, v_win, win_len
 
 
 _ORIG_WINDOW = O.attend_gqa_window
+_ORIG_CAUSAL = O.attend_gqa_causal
+
+
+def _causal_off_by_one(q, k_hat, v_hat, lengths, scale):
+    # each query also sees the next position
+    longer = [min(int(n) + 1, k_hat.shape[2]) for n in lengths]
+    return _ORIG_CAUSAL(q, k_hat, v_hat, longer, scale)
+
+
+def _causal_rows_reversed(q, k_hat, v_hat, lengths, scale):
+    # query i takes the limit of query Lq - 1 - i
+    return _ORIG_CAUSAL(q[:, :, ::-1], k_hat, v_hat, lengths, scale)[:, :, ::-1]
 
 
 MUTATIONS = {
@@ -186,6 +198,8 @@ MUTATIONS = {
     "window_scale_dropped": [("attend_gqa_window", _window_scale_dropped)],
     "window_length_ignored": [("attend_gqa_window", _window_length_ignored)],
     "window_replaces_packed_tail": [("attend_gqa_window", _window_before_packed_length)],
+    "causal_sees_one_more_key": [("attend_gqa_causal", _causal_off_by_one)],
+    "causal_rows_reversed": [("attend_gqa_causal", _causal_rows_reversed)],
 }
 
 

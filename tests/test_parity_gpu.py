@@ -478,3 +478,88 @@ def test_decode_g8_zero_and_window(sm, bits):
     assert np.all(o == 0.0)
     kw, vw, wl = _window(2, 2, 16, 128, [9, 16], seed=73)
     _check_window(sm, q, k, v, lens, kw, vw, wl, bits, 8, 1.0)
+
+
+# ---------------------------------------------------------------------------
+# causal multi-query attention (kvq_attend_causal)
+# ---------------------------------------------------------------------------
+
+def _check_causal(sm, q, k, v, lens, bits, group, scale, q_dtype=torch.bfloat16, splits=0):
+    """kvq_attend_causal against the oracle's causal rows on the decoded cache,
+    within 2e-3 * max|V_hat| of the head plus the bf16 output's own rounding
+    (a row near the start of a sequence reads few keys, so |O| can approach
+    max|V_hat|)."""
+    b_, hq, lq, d = q.shape
+    hkv = k.shape[1]
+    cache = pack_gpu(sm, k, v, bits, group)
+    qd = to_dev(q, q_dtype)
+    out = sm.attend(qd, cache, to_dev(lens, torch.int32), scale, splits=splits, causal=True)
+    sm.check()
+    o = out.float().cpu().numpy()
+    k_hat, v_hat = np.zeros_like(k), np.zeros_like(v)
+    for b in range(b_):
+        for h in range(hkv):
+            k_hat[b, h] = O.unpack_matrix(O.pack_k(k[b, h], bits, group))
+            v_hat[b, h] = O.unpack_matrix(O.pack_v(v[b, h], bits, group))
+    want = O.attend_gqa_causal(qd.float().cpu().numpy(), k_hat, v_hat, lens, scale)
+    grp = hq // hkv
+    for b in range(b_):
+        for h in range(hq):
+            tol = 2e-3 * float(np.abs(v_hat[b, h // grp, :lens[b]]).max())
+            err = np.abs(o[b, h] - want[b, h])
+            if q_dtype == torch.bfloat16:
+                err = err - np.abs(want[b, h]) * 2.0 ** -8
+            worst = float(err.max())
+            assert np.isfinite(o[b, h]).all() and worst <= tol, f"b{b} h{h}: {worst:.3e} > {tol:.3e}"
+    return o
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("lq", [32, 64])
+def test_causal_chunk(sm, bits, lq):
+    """Tensor-core chunk kernel with the causal mask: the last rows of a
+    block see part of it, some rows see no key of a split's first blocks,
+    lengths ending inside a block, one barely longer than the chunk."""
+    q, k, v, lens = _gqa_case(3, 8, 2, 700, 128, [700, 300, lq + 13], lq=lq, seed=80 + bits + lq, bits=bits)
+    cache = pack_gpu(sm, k, v, bits, 32)
+    assert sm.kernel_name(cache, 8, lq).startswith("chunk")
+    for splits in (0, 1, 5):
+        _check_causal(sm, q, k, v, lens, bits, 32, 1.0, splits=splits)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (8, 8)])
+def test_causal_generic(sm, bits, group):
+    """Generic kernel (D 64, five query rows, f32 Q) with the causal mask;
+    one sequence exactly Lq long (its first row reads one key)."""
+    q, k, v, lens = _gqa_case(3, 4, 2, 200, 64, [200, 37, 5], lq=5, seed=82, bits=bits)
+    for splits in (0, 3):
+        _check_causal(sm, q, k, v, lens, bits, group, 0.125, q_dtype=torch.float32, splits=splits)
+
+
+def test_causal_one_row_is_plain(sm):
+    """One query row at the last position sees every key: the causal call
+    equals the plain one bit for bit."""
+    q, k, v, lens = _gqa_case(2, 8, 2, 300, 128, [300, 157], seed=84)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    qd, ld = to_dev(q, torch.bfloat16), to_dev(lens, torch.int32)
+    a = sm.attend(qd, cache, ld, 1.0)
+    b = sm.attend(qd, cache, ld, 1.0, causal=True)
+    sm.check()
+    assert torch.equal(a, b)
+
+
+def test_causal_short_length(sm):
+    """A sequence shorter than the chunk: reported, its rows without a
+    visible key are zeros, every other row finite and correct."""
+    q, k, v, _ = _gqa_case(2, 4, 2, 64, 64, [64, 64], lq=6, seed=85)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device=DEV)
+    lens = torch.tensor([64, 3], dtype=torch.int32, device=DEV)
+    sm.attend(to_dev(q), cache, lens, 0.125, out=out, causal=True)
+    with pytest.raises(sm.KVQError) as e:
+        sm.check()
+    assert e.value.name == "KVQ_ERR_LENGTH"
+    o = out.cpu().numpy()
+    assert np.isfinite(o).all()
+    assert np.all(o[1, :, :3] == 0)            # rows 0..2 of sequence 1 see no key
+    sm.check()
