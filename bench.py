@@ -301,7 +301,8 @@ def run_kvq(args, rank, world, local_rank):
     # --window W: the last W tokens of each sequence stay unquantized (bf16)
     # in a recent-token window; the packed cache holds the tokens before them
     W_win = int(args.window)
-    append = uniform and not W_win
+    causal = bool(args.causal)
+    append = uniform and not W_win and not causal
     # the step's append: the K group(s) holding the new tokens (re-packed from a
     # float32 recent-token window) and the new tokens' V rows; only when every
     # sequence has the same length, since one kvq_pack call covers one range
@@ -343,7 +344,7 @@ def run_kvq(args, rank, world, local_rank):
         if W_win:
             K.attend_window(qd, c, lens, kwin, vwin, wlens, 1.0, out=out, workspace=ws)
         else:
-            K.attend(qd, c, lens, 1.0, out=out, workspace=ws)
+            K.attend(qd, c, lens, 1.0, out=out, workspace=ws, causal=causal)
     torch.cuda.synchronize()
     K.check(dev)
 
@@ -439,7 +440,7 @@ def run_kvq(args, rank, world, local_rank):
         if W_win:
             K.attend_window(q_in[j], c, lens, kwin, vwin, wlens, 1.0, out=o_dev[j], workspace=ws)
         else:
-            K.attend(q_in[j], c, lens, 1.0, out=o_dev[j], workspace=ws)
+            K.attend(q_in[j], c, lens, 1.0, out=o_dev[j], workspace=ws, causal=causal)
         done[j].record(stream)
 
     def e2e_copies(i, n, ready, done, out_read):
@@ -497,7 +498,11 @@ def run_kvq(args, rank, world, local_rank):
     else:
         abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g, lq=Lq)
     step_bytes = abytes + (append_bytes(B, H_kv, D, N - t0, Lq, bits, g) if append else 0)
-    attend_flops = 4 * H_q * Lq * D * int(np.sum(lens_np.astype(np.int64)))
+    if causal:
+        # row i of a chunk reads L - Lq + i + 1 keys
+        attend_flops = 4 * H_q * D * int(sum(Lq * (int(n) - Lq) + Lq * (Lq + 1) // 2 for n in lens_np))
+    else:
+        attend_flops = 4 * H_q * Lq * D * int(np.sum(lens_np.astype(np.int64)))
     ms_max, e2e_max = max_over_ranks([ms, e2e_ms], world, dev)
 
     res = None
@@ -530,8 +535,9 @@ def run_kvq(args, rank, world, local_rank):
                        "step": ("append (re-pack the K group(s) of the new tokens, pack their V rows) + attend"
                                 if append else
                                 f"attend over the packed tokens and a {W_win}-token bf16 window" if W_win else
+                                "causal attend (the Lq rows are each sequence's last positions)" if causal else
                                 "attend (per-sequence lengths; no shared append range)"),
-                       "window": W_win,
+                       "window": W_win, "causal": causal,
                        "l2": f"inputs larger than L2: 2 packed caches of {caches[0].nbytes() / 1e6:.0f} MB used in turn",
                        "parallelism": f"independent batch per GPU x{world}",
                        "attend_kernel": kname, "step_bytes": step_bytes,
@@ -546,7 +552,7 @@ def run_kvq(args, rank, world, local_rank):
                          "algorithmic_bytes_per_launch": abytes,
                          "algorithmic_flops_per_launch": attend_flops,
                          "attend_gbs": round(abytes / (att_ms * 1e-3) / 1e9, 1),
-                         "traffic": recorded_traffic(src, workload, bits, g, W_win)},
+                         "traffic": recorded_traffic(src, workload, bits, g, W_win or int(causal))},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_max / args.steps * 1e3, 3),
                     "pipeline": "inputs copied on a second stream into two alternating device sets, "
@@ -573,6 +579,9 @@ def main():
                     help="code width (default: the workload's, 4 for the chunk workload)")
     ap.add_argument("--group", type=int, choices=[8, 32], default=0,
                     help="scale group size (default: the workload's, 32)")
+    ap.add_argument("--causal", action="store_true",
+                    help="causal rows (kvq_attend_causal): the Lq query rows are each sequence's last "
+                         "positions; for the multi-query chunk workload")
     ap.add_argument("--window", type=int, default=0,
                     help="keep the last W tokens of each sequence unquantized (bf16) in a recent-token "
                          "window (kvq_attend_window); 0 = none")
@@ -631,7 +640,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     res, data = run_kvq(args, rank, world, local_rank)
-    if rank == 0 and not args.no_cpu_baseline and not args.window:
+    if rank == 0 and not args.no_cpu_baseline and not args.window and not args.causal:
         q, k, v, lens, meta = data
         nb, ts, heads = cpu_oracle_rate(q, k, v, lens, meta, args.cpu_heads, repeats=3, min_seconds=10.0)
         rate = nb / statistics.median(ts) / 1e9
