@@ -1,5 +1,5 @@
-// Tuned decode attention: D = 128, 4-bit codes, groups of 32, four query
-// heads per KV head (GQA), one query row per sequence.
+// Tuned decode attention: D = 128, 4- or 8-bit codes, groups of 32 or 8,
+// four query heads per KV head (GQA), one query row per sequence.
 //
 // What it computes is the block rule of "Block KV decoding: less workspace,
 // more time" (huhohoo.com/en/docs/llm/kv-block-decode-cost, section "Do not
@@ -12,12 +12,14 @@
 // ------------------
 // * The concatenated (b, h, 32-token block) list is split evenly over
 //   workers, one worker per warp pair (CTAs x pairs per CTA), each with a
-//   contiguous range; a 32-token block is exactly one K group, so one K scale
-//   row serves the whole block.  After the prologue no barrier spans more
+//   contiguous range; a 32-token block is exactly one K group at g32 (one K
+//   scale row serves the whole block) and four at g8 (each of the four lane
+//   groups of a warp takes one).  After the prologue no barrier spans more
 //   than a pair: every pair runs at its own pace.
 // * Each pair runs one pipeline of bulk copies (cp.async.bulk, completion
 //   counted on an mbarrier) carrying, per block, 32 tokens of K codes and V
-//   codes, the block's K scale row (512 B) and the tokens' V scales (512 B).
+//   codes, the block's K scale row(s) (512 B at g32, 2 KB at g8) and the
+//   tokens' V scales (512 B at g32, 2 KB at g8).
 //   - The S-warp (scores) keeps the segment's q in shared memory, folds the
 //     K scales into it once per block, unpacks K once for all four heads and
 //     writes per-lane partial scores; it also refills the pipeline.
@@ -342,7 +344,8 @@ __device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H
 }
 
 // Lane 0 arms the stage's barrier with the block's byte count and issues the
-// four copies: K codes, V codes, the K scale row and the V scales.
+// four copies: K codes, V codes, the K scale rows of the block's groups
+// holding valid tokens, and the V scales.
 template <int BITS, int GRP>
 __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS, GRP>& ps, int stage, int b,
                                             int h, int j, const int* slen) {
