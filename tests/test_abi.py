@@ -116,3 +116,44 @@ def test_workspace_size_grows_with_splits():
     a = K.lib.kvq_workspace_size(ctypes.byref(c), 8, 1, 8)
     b = K.lib.kvq_workspace_size(ctypes.byref(c), 8, 1, 64)
     assert 0 < a < b
+
+
+def test_window_argument_rules():
+    """kvq_attend_window rejects bad window arguments on the host (every call
+    here fails before a launch), and its workspace holds one more slot per
+    (b, h) than kvq_attend's."""
+    c = _cache()
+    plain = K.lib.kvq_workspace_size(ctypes.byref(c), 4, 1, 0)
+    need = K.lib.kvq_workspace_size_window(ctypes.byref(c), 4, 1, 0)
+    assert need > plain > 0
+
+    def call(kw=0x6000, vw=0x7000, wdt=K.KVQ_BF16, wl=0x8000, wcap=16, w=0x5000, wsb=need, lens=0x3000, hq=4):
+        return K.lib.kvq_attend_window(0x1000, K.KVQ_BF16, ctypes.byref(c), lens, kw, vw, wdt, wl, wcap, hq, 1,
+                                       1.0, 0x4000, w, wsb, 0, None)
+
+    assert call(wdt=3) == 1                      # window dtype
+    assert call(wcap=0) == 1                     # no window capacity
+    assert call(kw=0) == 1 and call(vw=0) == 1 and call(wl=0) == 1
+    assert call(hq=3) == 1
+    assert call(kw=0x6001) == 3                  # bf16 window misaligned
+    assert call(vw=0x7001, wdt=K.KVQ_F32) == 3
+    assert call(wl=0x8002) == 3
+    assert call(wsb=plain) == 4                  # the plain workspace is too small
+    assert call(w=0) == 4
+    assert call(w=0x5008) == 3
+
+
+def test_causal_argument_rules():
+    """kvq_attend_causal takes kvq_attend's arguments and rules."""
+    c = _cache()
+
+    def call(hq=4, lq=4, lens=0x3000, w=0x5000, wsb=1 << 30, dt=K.KVQ_BF16):
+        return K.lib.kvq_attend_causal(0x1000, dt, ctypes.byref(c), lens, hq, lq, 1.0, 0x4000, w, wsb, 0, None)
+
+    assert call(hq=3) == 1
+    assert call(lq=0) == 1
+    assert call(dt=3) == 1
+    assert call(lens=0) == 1
+    assert call(lens=0x3002) == 3
+    assert call(w=0) == 4
+    assert call(wsb=16) == 4
