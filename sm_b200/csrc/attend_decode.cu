@@ -72,6 +72,13 @@ struct Tr {
   static constexpr int kKsRows = 32 / GRP;          // K scale rows (groups) per 32-token block
   static constexpr int kVs = 128 / GRP;             // V scales per token
   static constexpr int kPvW = GRP == 32 ? 20 : 4;   // floats per token row of the p table
+  // How the pipeline refills.  Split: the S-warp streams each stage's K half
+  // and the V-warp its V half, each refilling right after its own last read
+  // (8-bit 114 -> 109 us, g8 slightly faster).  Whole: the S-warp refills
+  // the whole stage once the V-warp has released it, which measured faster
+  // at 4-bit g32 (91.8 us against 94.7 or 100.9 us split), where the
+  // 128-register budget leaves no room for a second copy cursor.
+  static constexpr bool kSplit = !(BITS == 4 && GRP == 32);
   // each channel's code f = 1 + code * eps sits in mantissa bits 15.. (even
   // 4-bit channels, every 8-bit channel: eps = 2^-8) or 19.. (odd 4-bit
   // channels: eps = 2^-4); corr = 1 + qmax * eps
@@ -100,8 +107,10 @@ struct PairSmem {
   float pv[kTB][Tr<BITS, GRP>::kPvW];  // g32: p' = p * s_v of token t, group g, head h at
                                       // [t][4g + h], four entries pad the row; g8: p of token
                                       // t, head h at [t][h] (the V scale goes on the codes)
-  unsigned long long full[Tr<BITS, GRP>::kS];    // copies landed
-  unsigned long long empty[Tr<BITS, GRP>::kS];   // V-warp done with the stage
+  unsigned long long full[Tr<BITS, GRP>::kS];    // split: the K half landed; whole: the stage landed
+  unsigned long long other[Tr<BITS, GRP>::kS];   // split: the V half landed; whole: the V-warp
+                                                 // released the stage
+  unsigned long long cursor[2][6];    // each warp's copy cursor (a Prod), lane 0's alone
   unsigned long long pfull[2];        // S-warp wrote part[i]
   unsigned long long pempty[2];       // V-warp read part[i]
 };
@@ -187,6 +196,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Orders this thread's earlier generic-proxy accesses of shared memory before
+// its later async-proxy (bulk copy) writes to it.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -343,7 +358,7 @@ __device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H
   return p;
 }
 
-// Lane 0 arms the stage's barrier with the block's byte count and issues the
+// Whole refill: lane 0 arms the stage's barrier with the block's byte count and issues the
 // four copies: K codes, V codes, the K scale rows of the block's groups
 // holding valid tokens, and the V scales.
 template <int BITS, int GRP>
@@ -365,6 +380,36 @@ __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS
            krows * kD * sizeof(float), bar);
   bulk_g2s(st.vs, p.v_scales + head * p.v_scales_head + static_cast<long long>(t0) * kVs,
            nv * kVs * 4, bar);
+}
+
+// Split refill: the S-warp streams the K half of each stage (K codes, the K scale rows of
+// the block's groups holding valid tokens) and the V-warp the V half (V
+// codes, V scales): each warp is the only reader of its half, so it refills
+// a stage as soon as its own reads of it are done.  Lane 0 arms the half's
+// barrier with its byte count and issues its two copies.
+template <int BITS, int GRP>
+__device__ __forceinline__ void issue_half(const DecodeParams& p, PairSmem<BITS, GRP>& ps, int stage, int b,
+                                           int h, int j, const int* slen, bool k_half) {
+  const long long head = static_cast<long long>(b) * p.H + h;
+  const int len = slen[b];
+  const int t0 = j * kTB;
+  const int nv = min(kTB, len - t0);
+  constexpr int kCb = Tr<BITS, GRP>::kCb;
+  constexpr int kVs = Tr<BITS, GRP>::kVs;
+  Stage<BITS, GRP>& st = ps.st[stage];
+  if (k_half) {
+    unsigned long long* bar = &ps.full[stage];
+    const int krows = (nv + GRP - 1) / GRP;                // K groups holding valid tokens
+    mbar_expect_tx(bar, static_cast<uint32_t>(kCb * nv + krows * kD * 4));
+    bulk_g2s(st.kc, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
+    bulk_g2s(st.ks, p.k_scales + head * p.k_scales_head + static_cast<long long>(t0 / GRP) * kD,
+             krows * kD * sizeof(float), bar);
+  } else {
+    unsigned long long* bar = &ps.other[stage];
+    mbar_expect_tx(bar, static_cast<uint32_t>((kCb + kVs * 4) * nv));
+    bulk_g2s(st.vc, p.v_codes + head * p.v_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
+    bulk_g2s(st.vs, p.v_scales + head * p.v_scales_head + static_cast<long long>(t0) * kVs, nv * kVs * 4, bar);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -393,7 +438,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
 #pragma unroll
     for (int s = 0; s < kS; ++s) {
       mbar_init(&ps.full[s], 1);
-      mbar_init(&ps.empty[s], 1);
+      mbar_init(&ps.other[s], 1);
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -413,8 +458,14 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
   if (cr.g0 >= cr.g1) return;
 
   Seg seg = first_seg(pre, p.B, H, cr);
+  constexpr bool kSplit = Tr<BITS, GRP>::kSplit;
+  // Whole refill: the S-warp's copy cursor, in registers.  Split refill:
+  // each warp's cursor lives in shared memory and only lane 0 touches it, so
+  // it takes no registers in the lanes' loops.
   Prod prod{seg, seg.jb, true};
   prod = prod_settle(prod, pre, p.B, H, cr);
+  static_assert(sizeof(Prod) <= sizeof(unsigned long long) * 6, "cursor slot");
+  Prod* cur = reinterpret_cast<Prod*>(ps.cursor[is_s ? 0 : 1]);
   // S-warp: q of a segment, loaded (lane + 32 r) before it is scaled into qs.
   // The first segment's loads go out before the first block copies so they
   // do not queue behind them.
@@ -435,15 +486,25 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       ps.qs[qs_index(i / kD, i % kD)] = qv[r] * qf;
     }
   };
-  if (is_s) {
-    load_q(seg);
+  if (is_s) load_q(seg);
+  if constexpr (kSplit) {
+    if (lane == 0) {
+      Prod pr = prod;
+      for (int s = 0; s < kS && pr.valid; ++s) {
+        issue_half<BITS, GRP>(p, ps, s, pr.seg.b, pr.seg.h, pr.j, slen, is_s);
+        ++pr.j;
+        pr = prod_settle(pr, pre, p.B, H, cr);
+      }
+      *cur = pr;
+    }
+  } else if (is_s) {
     for (int s = 0; s < kS && prod.valid; ++s) {
       if (lane == 0) issue_block<BITS, GRP>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
       ++prod.j;
       prod = prod_settle(prod, pre, p.B, H, cr);
     }
-    store_q();
   }
+  if (is_s) store_q();
 
   uint32_t k = 0;                                        // blocks this pair has consumed
   bool first = true;
@@ -516,13 +577,25 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
         __syncwarp();
         if (lane == 0) mbar_arrive(&ps.pfull[pb]);
 
-        // refill the stage of the previous block once the V-warp has released it
-        if (k > 0 && prod.valid) {
+        if constexpr (kSplit) {
+          // this warp has read the stage's K half for the last time: refill
+          // it with the block kS ahead
+          if (lane == 0) {
+            Prod pr = *cur;
+            if (pr.valid) {
+              fence_proxy_async();
+              issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, true);
+              ++pr.j;
+              *cur = prod_settle(pr, pre, p.B, H, cr);
+            }
+          }
+        } else if (k > 0 && prod.valid) {
+          // refill the stage of the previous block once the V-warp has
+          // released it: its reads of the stage happen before its arrive on
+          // `other`, which this wait acquires, so the copy cannot overtake them
           const uint32_t kp = k - 1;
           const int sp = static_cast<int>(kp % kS);
-          // the V-warp's reads of the stage happen before its arrive on
-          // `empty`, which this wait acquires: the copy cannot overtake them
-          wait_bar(&ps.empty[sp], (kp / kS) & 1u, p.err);
+          wait_bar(&ps.other[sp], (kp / kS) & 1u, p.err);
           if (lane == 0) issue_block<BITS, GRP>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
           ++prod.j;
           prod = prod_settle(prod, pre, p.B, H, cr);
@@ -544,7 +617,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
-        wait_bar(&ps.full[stage], (k / kS) & 1u, p.err);
+        wait_bar(kSplit ? &ps.other[stage] : &ps.full[stage], (k / kS) & 1u, p.err);
         wait_bar(&ps.pfull[pb], (k >> 1) & 1u, p.err);
         const Stage& st = ps.st[stage];
         const int nvalid = min(kTB, len - j * kTB);
@@ -635,7 +708,20 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
             for (int i = 0; i < 8; ++i) u[hh][i] = fma2(pp[hh], f[i], u[hh][i]);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ps.empty[stage]);
+        if constexpr (kSplit) {
+          // this warp has read the stage's V half for the last time: refill it
+          if (lane == 0) {
+            Prod pr = *cur;
+            if (pr.valid) {
+              fence_proxy_async();
+              issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, false);
+              ++pr.j;
+              *cur = prod_settle(pr, pre, p.B, H, cr);
+            }
+          }
+        } else if (lane == 0) {
+          mbar_arrive(&ps.other[stage]);               // the S-warp may refill the stage
+        }
       }
 
       // the pair's state for the segment: z summed over the token lanes, u
