@@ -23,6 +23,14 @@ summed over all ranks and divided by the max over ranks.
 ``--impl reference`` times the CPU oracle instead (NumPy, on this host's
 cores), on a bounded sample of the same workload, and reports the same
 metric.
+
+Studies of the kvq arm (not the headline): ``--workload`` long_context or
+chunk, ``--bits 8``, ``--group 8``, ``--window W`` (the last W tokens of each
+sequence kept unquantized, kvq_attend_window) and ``--causal`` (the chunk's
+rows are each sequence's last positions, kvq_attend_causal).  ``e2e`` goes
+through the Python API with every step's inputs copied in from pinned host
+memory and its output read back, the copies on a second stream so that the
+next step's inputs arrive while a step computes.
 """
 
 from __future__ import annotations
@@ -594,6 +602,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
+        if args.window or args.causal:
+            ap.error("--window and --causal are studies of the kvq arm; the reference arm times the "
+                     "oracle on the plain workload")
         if rank != 0:
             return 0
         q, k, v, lens, meta = W.gqa_case(args.workload, SEED)

@@ -9,6 +9,9 @@ is no fallback of any kind.
     cache = sm_b200.PackedCache(B, H_kv, N_cap, D, bits=4, group=32)
     sm_b200.pack(K, V, cache)                     # K, V [B, H_kv, T, D] fp32/bf16
     O = sm_b200.attend(Q, cache, lengths, scale)  # Q [B, H_q, Lq, D] fp32/bf16
+    O = sm_b200.attend(Q, cache, lengths, scale, causal=True)   # rows = last Lq positions
+    O = sm_b200.attend_window(Q, cache, lengths, K_win, V_win, win_lengths, scale)
+                                                  # packed tokens, then an unquantized window
 """
 
 from __future__ import annotations
