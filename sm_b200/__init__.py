@@ -123,7 +123,9 @@ class PackedCache:
     """Device memory of one packed cache, allocated through torch.
 
     k_codes / v_codes are uint8, k_scales / v_scales float32, each flat and
-    laid out as ``include/kvq.h`` describes."""
+    laid out as ``include/kvq.h`` describes.  Write into them in place if
+    needed, but do not rebind them: the C struct the calls pass is built
+    once from their addresses."""
 
     def __init__(self, B: int, H_kv: int, N_cap: int, D: int, bits: int = 4, group: int = 32,
                  device="cuda"):
