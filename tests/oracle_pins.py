@@ -217,6 +217,27 @@ def pin_17_over_3():
     assert abs(O.attend_dense(q, k, v, 1.0)[0, 0] - 17 / 3) < 1e-14
 
 
+def pin_17_over_3_window_and_causal():
+    """The pages' worked example through the two later paths.  Window: the
+    first two keys packed (decoded values given as they are), the third in
+    the window -- one softmax over all three gives 17/3.  Causal: three query
+    rows at positions 0, 1, 2 read one, two and three keys, giving the value
+    2, the first stop's 10/3 and the final 17/3."""
+    kv, _ = read_golden("online_softmax_17_3.txt")
+    s = [_num(t) for t in kv["scores"].split()]
+    vals = [_num(t) for t in kv["values"].split()]
+    k = np.array(s)[None, None, :, None]            # [B, H, N, D] with D = 1
+    v = np.array(vals)[None, None, :, None]
+    q1 = np.ones((1, 1, 1, 1))
+    win = O.attend_gqa_window(q1, k[:, :, :2], v[:, :, :2], [2], k[:, :, 2:], v[:, :, 2:], [1], 1.0)
+    assert abs(win[0, 0, 0, 0] - _num(kv["stop2_out"])) < 1e-14
+    q3 = np.ones((1, 1, 3, 1))
+    rows = O.attend_gqa_causal(q3, k, v, [3], 1.0)[0, 0, :, 0]
+    assert abs(rows[0] - vals[0]) < 1e-15
+    assert abs(rows[1] - _num(kv["stop1_out"])) < 1e-14
+    assert abs(rows[2] - _num(kv["stop2_out"])) < 1e-14
+
+
 def block_average(q, k, v, scale, block):
     """The wrong baseline the pages warn about: softmax each block on its own,
     then average the block outputs with equal weight."""
@@ -415,5 +436,5 @@ ALL_PINS = [
     pin_eight_bit, pin_ledger, pin_workspace_sizes, pin_17_over_3,
     pin_negative_example, pin_dense_vs_blocked, pin_bruteforce,
     pin_large_scores_stay_finite, pin_merge_partials, pin_gqa_and_lengths, pin_window,
-    pin_causal,
+    pin_causal, pin_17_over_3_window_and_causal,
 ]
