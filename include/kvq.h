@@ -56,7 +56,8 @@ extern "C" {
 typedef enum {
   KVQ_OK = 0,
   KVQ_ERR_ARG = 1,          /* bad bits/group/shape/dtype, H_q % H_kv != 0, NULL pointer */
-  KVQ_ERR_LENGTH = 2,       /* a sequence length <= 0 or > N_cap (device-detected: kvq_check) */
+  KVQ_ERR_LENGTH = 2,       /* a sequence length outside its valid range: 1..N_cap, or as the
+                               window and causal calls state (device-detected: kvq_check) */
   KVQ_ERR_ALIGN = 3,        /* a cache array or workspace not 16-byte aligned */
   KVQ_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than kvq_workspace_size() */
   KVQ_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute query) */

@@ -299,7 +299,7 @@ const char* kvq_strerror(kvq_status status) {
   switch (status) {
     case KVQ_OK: return "ok";
     case KVQ_ERR_ARG: return "invalid argument";
-    case KVQ_ERR_LENGTH: return "sequence length outside 1..N_cap";
+    case KVQ_ERR_LENGTH: return "sequence length outside its valid range (1..N_cap, or a window or causal rule)";
     case KVQ_ERR_ALIGN: return "pointer not suitably aligned";
     case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
     case KVQ_ERR_CUDA: return "CUDA runtime error";
