@@ -358,9 +358,9 @@ __device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H
   return p;
 }
 
-// Whole refill: lane 0 arms the stage's barrier with the block's byte count and issues the
-// four copies: K codes, V codes, the K scale rows of the block's groups
-// holding valid tokens, and the V scales.
+// Whole refill: lane 0 arms the stage's barrier with the block's byte count
+// and issues the four copies: K codes, V codes, the K scale rows of the
+// block's groups holding valid tokens, and the V scales.
 template <int BITS, int GRP>
 __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS, GRP>& ps, int stage, int b,
                                             int h, int j, const int* slen) {
@@ -382,11 +382,11 @@ __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS
            nv * kVs * 4, bar);
 }
 
-// Split refill: the S-warp streams the K half of each stage (K codes, the K scale rows of
-// the block's groups holding valid tokens) and the V-warp the V half (V
-// codes, V scales): each warp is the only reader of its half, so it refills
-// a stage as soon as its own reads of it are done.  Lane 0 arms the half's
-// barrier with its byte count and issues its two copies.
+// Split refill: the S-warp streams the K half of each stage (K codes, the K
+// scale rows of the block's groups holding valid tokens) and the V-warp the
+// V half (V codes, V scales): each warp is the only reader of its half, so
+// it refills a stage as soon as its own reads of it are done.  Lane 0 arms
+// the half's barrier with its byte count and issues its two copies.
 template <int BITS, int GRP>
 __device__ __forceinline__ void issue_half(const DecodeParams& p, PairSmem<BITS, GRP>& ps, int stage, int b,
                                            int h, int j, const int* slen, bool k_half) {
