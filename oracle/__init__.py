@@ -22,10 +22,10 @@ Every function names the page and section it follows.  Pages:
   -- softmax(QK^T/sqrt(d_k))V, GQA sharing, mask rules, the 17/3 example.
 
 Parity status: every public function is pinned by ``tests/test_oracle_pins.py``
-against values the pages print, closed forms, brute force or error bounds,
-except ``rel_l2_error`` magnitudes, which are a soft band (the pages' random
-inputs cannot be regenerated) -- that band is "parity unpinned" at the value
-level.
+against values the pages print, closed forms, brute force or error bounds
+(``rel_l2_error`` by closed forms); only the magnitudes of the pages' error
+table are a soft band (their random inputs cannot be regenerated) -- that
+band is "parity unpinned" at the value level.
 """
 
 from .kvq_oracle import (  # noqa: F401

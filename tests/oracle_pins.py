@@ -408,6 +408,23 @@ def pin_causal():
     assert np.max(np.abs(one - O.attend_gqa(q[:, :, :1], k, v, lens, 0.8))) < 1e-12
 
 
+def pin_rel_l2_definition():
+    """The error measure itself, by closed forms: zero for identical arrays,
+    1 for twice the reference, |e| / |x| for an error orthogonal to the
+    reference (here 3-4-5: |e| = 5 against |x| = 10), taken over the whole
+    array, not per row."""
+    x = np.array([[6.0, 0.0], [0.0, 8.0]])
+    assert O.rel_l2_error(x, x) == 0.0
+    assert abs(O.rel_l2_error(2 * x, x) - 1.0) < 1e-15
+    e = np.array([[0.0, 3.0], [4.0, 0.0]])
+    assert abs(O.rel_l2_error(x + e, x) - 0.5) < 1e-15
+    # whole-array norm: a per-row mean would give (3/6 + 4/8) / 2 = 0.5 too, so
+    # use rows of different scale to tell them apart
+    y = np.array([[1.0, 0.0], [0.0, 100.0]])
+    f = np.array([[0.0, 1.0], [0.0, 0.0]])
+    assert abs(O.rel_l2_error(y + f, y) - 1.0 / math.sqrt(10001.0)) < 1e-15
+
+
 def pin_rel_l2_band():
     """Soft check (parity unpinned at the value level): the mean relative L2
     output error on the six clean inputs lands near the pages' table, and the
@@ -436,5 +453,5 @@ ALL_PINS = [
     pin_eight_bit, pin_ledger, pin_workspace_sizes, pin_17_over_3,
     pin_negative_example, pin_dense_vs_blocked, pin_bruteforce,
     pin_large_scores_stay_finite, pin_merge_partials, pin_gqa_and_lengths, pin_window,
-    pin_causal, pin_17_over_3_window_and_causal,
+    pin_causal, pin_17_over_3_window_and_causal, pin_rel_l2_definition,
 ]

@@ -166,6 +166,18 @@ def _window_before_packed_length(q, k_hat, v_hat, lengths, k_win, v_win, win_len
     return _ORIG_WINDOW(q, k_hat, v_hat, cut, k_win, v_win, win_lengths, scale)
 
 
+def _rel_l2_per_row(out, ref):
+    out = np.atleast_2d(np.asarray(out, np.float64))
+    ref = np.atleast_2d(np.asarray(ref, np.float64))
+    return float(np.mean(np.linalg.norm(out - ref, axis=-1) / np.linalg.norm(ref, axis=-1)))
+
+
+def _rel_l1(out, ref):
+    out = np.asarray(out, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return float(np.abs(out - ref).sum() / np.abs(ref).sum())
+
+
 _ORIG_WINDOW = O.attend_gqa_window
 _ORIG_CAUSAL = O.attend_gqa_causal
 
@@ -200,6 +212,8 @@ MUTATIONS = {
     "window_replaces_packed_tail": [("attend_gqa_window", _window_before_packed_length)],
     "causal_sees_one_more_key": [("attend_gqa_causal", _causal_off_by_one)],
     "causal_rows_reversed": [("attend_gqa_causal", _causal_rows_reversed)],
+    "rel_l2_per_row_mean": [("rel_l2_error", _rel_l2_per_row)],
+    "rel_l1_instead_of_l2": [("rel_l2_error", _rel_l1)],
 }
 
 
