@@ -52,5 +52,4 @@ from .kvq_oracle import (  # noqa: F401
     attend_gqa_window,
     attend_gqa_causal,
     rel_l2_error,
-    pack_cache,
 )

@@ -500,11 +500,3 @@ def rel_l2_error(out: np.ndarray, ref: np.ndarray) -> float:
     ref = np.asarray(ref, np.float64)
     return float(np.linalg.norm(out - ref) / np.linalg.norm(ref))
 
-
-def pack_cache(k: np.ndarray, v: np.ndarray, bits: int, group: int):
-    """Pack every (b, h) matrix of [B, H, N, D] K and V independently.
-    Returns nested lists [b][h] of (PackedMatrix K, PackedMatrix V)."""
-    k = np.asarray(k, np.float32)
-    v = np.asarray(v, np.float32)
-    return [[(pack_k(k[b, h], bits, group), pack_v(v[b, h], bits, group))
-             for h in range(k.shape[1])] for b in range(k.shape[0])]

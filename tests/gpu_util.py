@@ -64,5 +64,38 @@ def oracle_rows(q_vals: np.ndarray, k: np.ndarray, v: np.ndarray, bits: int, gro
     return want, pk, pv, vh[:length]
 
 
+def bf16_rounding_gap(out_bf16: np.ndarray, want: np.ndarray) -> np.ndarray:
+    """Distance from each oracle value to the set of reals that round (to
+    nearest, ties to even) to the kernel's bf16 output.  The kernel computes
+    in float32 and rounds once when it stores O; this is the smallest error
+    its float32 result can have had, so ``gap <= tol`` is exactly "some
+    float32 result within tol of the oracle gives this output" -- the output
+    rounding is allowed for, and nothing more.
+
+    out_bf16: the output's values as float32 (each exactly a bf16 value)."""
+    o = np.asarray(out_bf16, np.float32)
+    w = np.asarray(want, np.float64)
+    a = np.abs(o)
+    bits = a.view(np.uint32)
+    assert np.all((bits & 0xFFFF) == 0), "not bf16 values"
+    up = (bits + 0x10000).view(np.float32).astype(np.float64) - a        # spacing above |o|
+    down_bits = np.where(bits >= 0x10000, bits - 0x10000, 0).astype(np.uint32)
+    down = a.astype(np.float64) - down_bits.view(np.float32).astype(np.float64)
+    down = np.where(bits == 0, up, down)                                 # +-0: symmetric
+    # half the spacing on the side of the oracle value, mirrored for o < 0
+    away = (w - o) * np.where(o < 0, -1.0, 1.0) > 0                     # oracle beyond |o|
+    half = np.where(away, up, down) / 2.0
+    return np.maximum(0.0, np.abs(w - o) - half)
+
+
+def check_rows_rounded(out_bf16: np.ndarray, want: np.ndarray, tol: float, what: str) -> float:
+    """A bf16 output against the float64 oracle: the oracle value must lie
+    within ``tol`` of the output's rounding interval (bf16_rounding_gap)."""
+    assert np.isfinite(out_bf16).all(), f"{what}: non-finite output"
+    worst = float(bf16_rounding_gap(out_bf16, want).max())
+    assert worst <= tol, f"{what}: max|err| beyond the output rounding {worst:.3e} > {tol:.3e}"
+    return worst
+
+
 def single_head_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)

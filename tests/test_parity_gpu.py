@@ -2,7 +2,7 @@
 2e-3 * max|V_hat| of the float64 oracle on the same decoded cache, on every
 workload shape -- the single-head grid, the 35 x 13 edge case, ragged GQA
 cases spanning several blocks and a tail, and the full-size decode,
-long-context and chunk workloads (sampled heads)."""
+long-context and chunk workloads (every head)."""
 
 from __future__ import annotations
 
@@ -14,8 +14,8 @@ import torch
 
 import oracle as O
 import workloads as W
-from tests.gpu_util import (DEV, assert_head_packed_equal, bf16_values, check_rows, oracle_rows,
-                            pack_gpu, single_head_scale, to_dev)
+from tests.gpu_util import (DEV, assert_head_packed_equal, bf16_values, check_rows, check_rows_rounded,
+                            oracle_rows, pack_gpu, single_head_scale, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -301,40 +301,40 @@ def test_bad_lengths_reported(sm):
 
 
 # ---------------------------------------------------------------------------
-# full-size workloads, sampled heads
+# full-size workloads, every head against the oracle
 # ---------------------------------------------------------------------------
 
-SAMPLE = [(0, 0), (5, 3), (17, 7), (31, 1)]
-
-
-def _full_case(sm, name, seed=0, bits=4, heads=SAMPLE, splits=0):
+def _full_case(sm, name, seed=0, bits=4, group=None, splits=0):
+    """The named workload at its full size, in the launch configuration the
+    bench times (automatic splits): every (b, h_kv) head's cache bytes and
+    output rows against the oracle.  Different heads take different paths
+    through the work plan (whole-segment output or partials and the merge,
+    worker boundaries at different blocks), so none is left out."""
     q, k, v, lens, meta = W.gqa_case(name, seed)
     q = bf16_values(q)
-    _check_gqa(sm, q, k, v, lens, bits, meta["group"], 1.0, splits=splits,
-               heads=[(b % meta["B"], h) for b, h in heads])
+    _check_gqa(sm, q, k, v, lens, bits, group or meta["group"], 1.0, splits=splits)
 
 
 def test_decode_gqa_full(sm):
     _full_case(sm, "decode_gqa")
 
 
-def test_decode_gqa_full_8bit(sm):
-    """The decode workload with 8-bit codes (the tuned decode kernel's 8-bit
-    form), sampled heads against the oracle."""
-    q, k, v, lens, meta = W.gqa_case("decode_gqa", 0)
-    q = bf16_values(q)
-    small = pack_gpu(sm, np.ascontiguousarray(k[:1, :, :64]), np.ascontiguousarray(v[:1, :, :64]), 8, meta["group"])
-    assert sm.kernel_name(small, meta["H_q"], 1).startswith("decode_gqa4")
-    _check_gqa(sm, q, k, v, lens, 8, meta["group"], 1.0, heads=SAMPLE)
+@pytest.mark.parametrize("bits,group", [(8, 32), (4, 8), (8, 8)])
+def test_decode_gqa_full_formats(sm, bits, group):
+    """The decode workload in the other code widths and group sizes of the
+    tuned decode kernel."""
+    small = sm.PackedCache(1, 8, 64, 128, bits, group, DEV)
+    assert sm.kernel_name(small, 32, 1).startswith("decode_gqa4")
+    _full_case(sm, "decode_gqa", bits=bits, group=group)
 
 
 def test_long_context_full(sm):
-    _full_case(sm, "long_context", heads=[(0, 0), (3, 5), (7, 7), (6, 2)])
+    _full_case(sm, "long_context")
 
 
 @pytest.mark.parametrize("bits", [4, 8])
 def test_chunk_full(sm, bits):
-    _full_case(sm, "chunk", bits=bits, heads=[(0, 0), (1, 5), (3, 7)])
+    _full_case(sm, "chunk", bits=bits)
 
 
 # ---------------------------------------------------------------------------
@@ -366,13 +366,13 @@ def _check_window(sm, q, k, v, lens, kw, vw, wl, bits, group, scale, q_dtype=tor
     for b in range(b_):
         vals = np.concatenate([v_hat[b, :, :lens[b]].ravel(), vwv[b, :, :wl[b]].ravel()])
         tol = 2e-3 * float(np.abs(vals).max())
-        # a bf16 output carries its own rounding, up to 2^-8 of the value: a
-        # row that follows one window key can sit near max|V| itself
-        err = np.abs(o[b] - want[b])
+        # a row that follows one window key can sit near max|V| itself, where
+        # one bf16 rounding of the output alone exceeds the tolerance: a bf16
+        # output is checked through its rounding interval
         if q_dtype == torch.bfloat16:
-            err = err - np.abs(want[b]) * 2.0 ** -8
-        worst = float(err.max())
-        assert np.isfinite(o[b]).all() and worst <= tol, f"b{b}: max|err| {worst:.3e} > {tol:.3e}"
+            check_rows_rounded(o[b], want[b], tol, f"b{b}")
+        else:
+            check_rows(o[b], want[b], vals, f"b{b}")
     return o
 
 
@@ -486,9 +486,10 @@ def test_decode_g8_zero_and_window(sm, bits):
 
 def _check_causal(sm, q, k, v, lens, bits, group, scale, q_dtype=torch.bfloat16, splits=0):
     """kvq_attend_causal against the oracle's causal rows on the decoded cache,
-    within 2e-3 * max|V_hat| of the head plus the bf16 output's own rounding
-    (a row near the start of a sequence reads few keys, so |O| can approach
-    max|V_hat|)."""
+    within 2e-3 * max|V_hat| of the head; a bf16 output through its rounding
+    interval (a row near the start of a sequence reads few keys, so |O| can
+    approach max|V_hat|, where one bf16 rounding alone exceeds the
+    tolerance)."""
     b_, hq, lq, d = q.shape
     hkv = k.shape[1]
     cache = pack_gpu(sm, k, v, bits, group)
@@ -505,12 +506,11 @@ def _check_causal(sm, q, k, v, lens, bits, group, scale, q_dtype=torch.bfloat16,
     grp = hq // hkv
     for b in range(b_):
         for h in range(hq):
-            tol = 2e-3 * float(np.abs(v_hat[b, h // grp, :lens[b]]).max())
-            err = np.abs(o[b, h] - want[b, h])
+            vh = v_hat[b, h // grp, :lens[b]]
             if q_dtype == torch.bfloat16:
-                err = err - np.abs(want[b, h]) * 2.0 ** -8
-            worst = float(err.max())
-            assert np.isfinite(o[b, h]).all() and worst <= tol, f"b{b} h{h}: {worst:.3e} > {tol:.3e}"
+                check_rows_rounded(o[b, h], want[b, h], 2e-3 * float(np.abs(vh).max()), f"b{b} h{h}")
+            else:
+                check_rows(o[b, h], want[b, h], vh, f"b{b} h{h}")
     return o
 
 
