@@ -226,6 +226,49 @@ class ClockSampler:
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
+def event_times_us(run, n: int, stream, between=None):
+    """Device times (µs) of n calls run(i), each bracketed by its own CUDA
+    events on `stream`.  between(i), if given, runs before call i outside
+    the events (an L2 flush)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        if between is not None:
+            between(i)
+        ev[i][0].record(stream)
+        run(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) * 1e3 for a, b in ev]
+
+
+def distribution(us):
+    """Median, p10 and p90 of a list of observations, and the list itself."""
+    a = np.asarray(us, np.float64)
+    return {"median": round(float(np.median(a)), 3), "p10": round(float(np.percentile(a, 10)), 3),
+            "p90": round(float(np.percentile(a, 90)), 3), "n": int(a.size),
+            "all": [round(float(x), 3) for x in a]}
+
+
+class L2Flush:
+    """Writes a buffer twice the size of L2 (at least 256 MB), outside any
+    timed region, so the next launch finds none of its inputs in L2."""
+
+    def __init__(self, dev):
+        import torch
+        l2 = 0
+        try:
+            l2 = int(torch.cuda.get_device_properties(dev).L2_cache_size)
+        except Exception:
+            pass
+        self.buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+        self.n = 0
+
+    def __call__(self, *_):
+        self.n += 1
+        self.buf.fill_(self.n & 0xFF)
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
@@ -356,8 +399,16 @@ def run_kvq(args, rank, world, local_rank):
     torch.cuda.synchronize()
     K.check(dev)
 
+    # one decode step per sequence (Lq = 1): kvq_decode_step re-packs the
+    # K group of the new token and packs its V row in one kernel, then
+    # attends; the multi-query chunk appends its Lq tokens with kvq_pack
+    decode_step = append and Lq == 1
+
     def step(i):
         c = caches[i & 1]
+        if decode_step:
+            K.decode_step(qd, c, lens, win_k, new_v, 1.0, out=out, workspace=ws)
+            return
         if append:
             K.pack(win_k, None, c, t0=t0)
             K.pack(None, new_v, c, t0=v0)
@@ -412,14 +463,12 @@ def run_kvq(args, rank, world, local_rank):
     K.check(dev)
     ms = start.elapsed_time(end)
 
-    # the attend kernel alone, same caches in turn, for the roofline
-    a_start, a_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a_start.record(stream)
-    for i in range(args.steps):
-        attend_graphs[i & 1][0].replay()
-    a_end.record(stream)
-    torch.cuda.synchronize()
-    attend_ms = [a_start.elapsed_time(a_end) / args.steps]
+    # the attend alone, for the roofline: at least 50 replays, each timed by
+    # its own events, the two caches in turn (each larger than L2)
+    n_att = max(50, args.steps)
+    attend_us = event_times_us(lambda i: attend_graphs[i & 1][0].replay(), n_att, stream)
+    attend_dist = distribution(attend_us)
+    attend_ms = [attend_dist["median"] / 1e3]
 
     # end-to-end through the public API (direct calls, no graphs): every step
     # copies its inputs from pinned host buffers and reads its output back,
@@ -442,6 +491,10 @@ def run_kvq(args, rank, world, local_rank):
         stream.wait_event(ready[j])
         if i >= 2:
             stream.wait_event(out_read[j])                # step i - 2's output has been read back
+        if decode_step:
+            K.decode_step(q_in[j], c, lens, k_in[j], v_in[j], 1.0, out=o_dev[j], workspace=ws)
+            done[j].record(stream)
+            return
         if append:
             K.pack(k_in[j], None, c, t0=t0)
             K.pack(None, v_in[j], c, t0=v0)
@@ -540,7 +593,9 @@ def run_kvq(args, rank, world, local_rank):
             "config": {"workload": workload, "B": B, "H_q": H_q, "H_kv": H_kv, "d_h": D,
                        "context": N if uniform else "per-sequence", "lengths_sum": int(np.sum(lens_np)),
                        "bits": bits, "group": g, "lq": Lq,
-                       "step": ("append (re-pack the K group(s) of the new tokens, pack their V rows) + attend"
+                       "step": ("kvq_decode_step: append (re-pack the K group of each sequence's new token, "
+                                "pack its V row; one kernel) + attend" if decode_step else
+                                "append (re-pack the K group(s) of the new tokens, pack their V rows) + attend"
                                 if append else
                                 f"attend over the packed tokens and a {W_win}-token bf16 window" if W_win else
                                 "causal attend (the Lq rows are each sequence's last positions)" if causal else
@@ -556,7 +611,9 @@ def run_kvq(args, rank, world, local_rank):
                          "frac": round(achieved / peak, 4),
                          "peak_source": ("bf16_tflops (burst) of " if tensor else "hbm_gbs of ") + peak_kind,
                          "kernel": f"kvq_attend ({kname})", "attend_us": round(att_ms * 1e3, 3),
-                         "timing": "attend-only CUDA-graph replays, same caches in turn",
+                         "attend_us_dist": attend_dist,
+                         "timing": f"median of {n_att} attend-only CUDA-graph replays, each timed by its own "
+                                   "events, the two caches in turn",
                          "algorithmic_bytes_per_launch": abytes,
                          "algorithmic_flops_per_launch": attend_flops,
                          "attend_gbs": round(abytes / (att_ms * 1e-3) / 1e9, 1),
@@ -572,6 +629,143 @@ def run_kvq(args, rank, world, local_rank):
     return res, (q_np, k_np, v_np, lens_np, meta)
 
 
+# ---------------------------------------------------------------------------
+# the other configurations: attend-only device times for the record
+# ---------------------------------------------------------------------------
+
+def capture_graph(K, fn, dev, stream):
+    """A CUDA graph of fn() (warmed once on a side stream) and the number of
+    library kernels it launches."""
+    import torch
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        fn()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    n0 = K.launch_count()
+    with torch.cuda.graph(g, stream=side):
+        fn()
+    torch.cuda.synchronize()
+    return g, K.launch_count() - n0
+
+
+def study_gqa(K, dev, stream, flush, workload: str, bits: int, n_rep: int = 50):
+    """Attend-only device time of a GQA workload at full size (one cache,
+    every replay after an L2 flush) with its roofline fraction: HBM bytes for
+    the decode shapes, bf16 tensor FLOPs for the multi-query chunk."""
+    import torch
+    q_np, k_np, v_np, lens_np, meta = W.gqa_case(workload, SEED)
+    B, H_q, H_kv, D, N, Lq, g = meta["B"], meta["H_q"], meta["H_kv"], meta["D"], meta["N"], meta["Lq"], meta["group"]
+    cache = K.PackedCache(B, H_kv, N, D, bits, g, dev)
+    kd = torch.from_numpy(k_np).to(dev)
+    vd = torch.from_numpy(v_np).to(dev)
+    K.pack(kd, vd, cache)
+    del kd, vd, k_np, v_np
+    qd = torch.from_numpy(q_np).to(dev).to(torch.bfloat16)
+    lens = torch.from_numpy(lens_np).to(dev)
+    out = torch.empty_like(qd)
+    ws = torch.empty(max(K.workspace_size(cache, H_q, Lq), 16), dtype=torch.uint8, device=dev)
+    graph, launches = capture_graph(K, lambda: K.attend(qd, cache, lens, 1.0, out=out, workspace=ws), dev, stream)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    d = distribution(event_times_us(lambda i: graph.replay(), n_rep, stream, between=flush))
+    K.check(dev)
+    med_s = d["median"] * 1e-6
+    abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g, lq=Lq)
+    flops = 4 * H_q * Lq * D * int(np.sum(lens_np.astype(np.int64)))
+    res = {"attend_us": d, "kernel": K.kernel_name(cache, H_q, Lq), "launches_per_attend": launches,
+           "bits": bits, "group": g, "B": B, "H_q": H_q, "H_kv": H_kv, "d_h": D, "lq": Lq,
+           "lengths_sum": int(np.sum(lens_np)), "algorithmic_bytes": abytes, "flops": flops,
+           "gbs": round(abytes / med_s / 1e9, 1)}
+    if Lq > 1:
+        peak, kind = measured_peaks("tensor")
+        tf = flops / med_s / 1e12
+        res.update({"tflops": round(tf, 2), "frac": round(tf / peak, 4), "bound": "tensor",
+                    "peak": peak, "peak_source": f"bf16_tflops (burst) of {kind}"})
+    else:
+        peak, kind = measured_peaks("hbm")
+        res.update({"frac": round(abytes / med_s / 1e9 / peak, 4), "bound": "hbm", "peak": peak,
+                    "peak_source": f"hbm_gbs of {kind}", "pct_of_8tbs": round(100 * abytes / med_s / 8e12, 2)})
+    del cache, qd, out, ws, graph
+    torch.cuda.empty_cache()
+    return res
+
+
+def study_single_head(K, dev, stream, flush, n_rep: int = 50):
+    """The single-head configurations (one head, 4 queries, D 32, N 128 and
+    512, every code width and group size): device µs of one attend, each
+    replay after an L2 flush.  They are launch-latency bound."""
+    import torch
+    out = {}
+    for n in (128, 512):
+        q, k, v = W.single_head(n, 32, 4, SEED, "clean")
+        for bits, g in W.FORMATS:
+            cache = K.PackedCache(1, 1, n, 32, bits, g, dev)
+            K.pack(torch.from_numpy(k[None, None]).to(dev), torch.from_numpy(v[None, None]).to(dev), cache)
+            qd = torch.from_numpy(q[None, None]).to(dev)
+            lens = torch.tensor([n], dtype=torch.int32, device=dev)
+            o = torch.empty_like(qd)
+            ws = torch.empty(max(K.workspace_size(cache, 1, 4), 16), dtype=torch.uint8, device=dev)
+            graph, _ = capture_graph(K, lambda: K.attend(qd, cache, lens, 1.0 / math.sqrt(32), out=o, workspace=ws),
+                                     dev, stream)
+            for _ in range(3):
+                graph.replay()
+            d = distribution(event_times_us(lambda i: graph.replay(), n_rep, stream, between=flush))
+            out[f"n{n}_b{bits}_g{g}"] = {"median": d["median"], "p10": d["p10"], "p90": d["p90"], "n": d["n"],
+                                         "kernel": K.kernel_name(cache, 1, 4)}
+    K.check(dev)
+    return out
+
+
+def oracle_single_head_protocol():
+    """The pages' CPU timing protocol on the oracle ("Block KV decoding: less
+    workspace, more time", section "CPU timing retains the negative result"):
+    the 18 single-head inputs (N 128 and 512, seeds 0-2, clean / early / late)
+    at 4-bit g32, three methods -- attention over the float32 cache, decode
+    everything then attend, decode and merge 32-token blocks -- each input
+    with 3 warm-up and 15 measured rounds in rotated method order; the
+    median µs per (N, method) over every observation, which are all kept."""
+    import oracle as O
+    scale = 1.0 / math.sqrt(32)
+    methods = {
+        "float32_cache": lambda q, k, v, pk, pv: O.attend_dense(q, k, v, scale),
+        "decode_all_then_attend": lambda q, k, v, pk, pv: O.attend_dense(q, O.unpack_matrix(pk),
+                                                                         O.unpack_matrix(pv), scale),
+        "decode_and_merge_blocks": lambda q, k, v, pk, pv: O.attend_blocked_packed(q, pk, pv, scale, 32),
+    }
+    names = list(methods)
+    obs = {(n, m): [] for n in (128, 512) for m in names}
+    for n, seed, dist in W.SINGLE_HEAD_GRID:
+        q, k, v = W.single_head(n, 32, 4, seed, dist)
+        pk, pv = O.pack_k(k, 4, 32), O.pack_v(v, 4, 32)
+        for r in range(3 + 15):
+            order = names[r % 3:] + names[:r % 3]
+            for m in order:
+                t = time.perf_counter()
+                methods[m](q, k, v, pk, pv)
+                dt = (time.perf_counter() - t) * 1e6
+                if r >= 3:
+                    obs[(n, m)].append(dt)
+    return {f"n{n}": {m: round(float(np.median(obs[(n, m)])), 1) for m in names} for n in (128, 512)} | {
+        "observations": sum(len(x) for x in obs.values()), "cores": blas_threads(),
+        "protocol": "18 inputs x 3 methods x 15 rounds (after 3 warm-ups), method order rotated each round, "
+                    "median per (N, method)"}
+
+
+def run_studies(K, dev, stream):
+    flush = L2Flush(dev)
+    res = {"timing": "attend-only CUDA-graph replays, each timed by its own events after an L2 flush"}
+    res["long_context"] = study_gqa(K, dev, stream, flush, "long_context", 4)
+    res["chunk_4bit"] = study_gqa(K, dev, stream, flush, "chunk", 4)
+    res["chunk_8bit"] = study_gqa(K, dev, stream, flush, "chunk", 8)
+    res["single_head_us"] = study_single_head(K, dev, stream, flush)
+    del flush
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -579,6 +773,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-studies", action="store_true",
+                    help="skip the attend-only timings of the other configurations (long context, chunk, "
+                         "single head) that the default run adds to its JSON line")
     ap.add_argument("--cpu-heads", type=int, default=256,
                     help="(b, h_kv) heads in the oracle's timed sample")
     ap.add_argument("--workload", choices=sorted(W.WORKLOADS), default=WORKLOAD,
@@ -651,6 +848,12 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     res, data = run_kvq(args, rank, world, local_rank)
+    plain = not args.window and not args.causal and not args.bits and not args.group
+    if rank == 0 and world == 1 and plain and args.workload == WORKLOAD and not args.no_studies:
+        dev = torch.device("cuda", local_rank)
+        res["studies"] = run_studies(__import__("sm_b200"), dev, torch.cuda.current_stream(dev))
+        if not args.no_cpu_baseline:
+            res["studies"]["single_head_oracle_host_us"] = oracle_single_head_protocol()
     if rank == 0 and not args.no_cpu_baseline and not args.window and not args.causal:
         q, k, v, lens, meta = data
         nb, ts, heads = cpu_oracle_rate(q, k, v, lens, meta, args.cpu_heads, repeats=3, min_seconds=10.0)

@@ -58,7 +58,8 @@ typedef enum {
   KVQ_ERR_ARG = 1,          /* bad bits/group/shape/dtype, H_q % H_kv != 0, NULL pointer */
   KVQ_ERR_LENGTH = 2,       /* a sequence length outside its valid range: 1..N_cap, or as the
                                window and causal calls state (device-detected: kvq_check) */
-  KVQ_ERR_ALIGN = 3,        /* a cache array or workspace not 16-byte aligned */
+  KVQ_ERR_ALIGN = 3,        /* a cache array, Q, O or the workspace not 16-byte aligned (or an
+                               input of kvq_pack not aligned to its element size) */
   KVQ_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than kvq_workspace_size() */
   KVQ_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute query) */
   KVQ_ERR_DEVICE = 6,       /* a kernel recorded an internal inconsistency */
@@ -100,6 +101,11 @@ typedef struct {
 KVQ_API kvq_status kvq_cache_sizes(int32_t bits, int32_t group, int32_t B, int32_t H_kv,
                            int32_t N_cap, int32_t D, size_t sizes[4]);
 
+/* Total bytes of the four arrays of `cache` (host; its pointers are not
+ * read): the sum of kvq_cache_sizes for its shape, 0 for an invalid shape or
+ * NULL. */
+KVQ_API size_t kvq_cache_bytes(const kvq_cache* cache);
+
 /*
  * Quantize and pack tokens [t0, t1) of every (b, h) into the cache.
  *   K, V     device, [B, H_kv, t1 - t0, D] in `in_dtype` (KVQ_F32 or
@@ -122,12 +128,13 @@ KVQ_API kvq_status kvq_pack(const void* K, const void* V, kvq_dtype in_dtype, in
 
 /*
  * Attention of Q over the packed cache.
- *   Q        device, [B, H_q, Lq, D] in q_dtype (KVQ_F32 or KVQ_BF16).
+ *   Q        device, [B, H_q, Lq, D] in q_dtype (KVQ_F32 or KVQ_BF16),
+ *            16-byte aligned.
  *   lengths  device int32 [B]: valid keys of each sequence, 1..N_cap.
  *   H_q      multiple of cache->H_kv.   Lq >= 1 query rows per sequence.
  *   scale    multiplies Q K^T before the softmax (1/sqrt(D) for unscaled Q,
  *            1 when Q already carries it).
- *   O        device, [B, H_q, Lq, D] in q_dtype.
+ *   O        device, [B, H_q, Lq, D] in q_dtype, 16-byte aligned.
  *   workspace, ws_bytes   device scratch for split partials, at least
  *            kvq_workspace_size(...) bytes, 16-byte aligned.  Its contents
  *            on entry do not matter; it must not be shared by calls that may
@@ -160,6 +167,41 @@ KVQ_API kvq_status kvq_attend_causal(const void* Q, kvq_dtype q_dtype, const kvq
                                      const int32_t* lengths, int32_t H_q, int32_t Lq, float scale,
                                      void* O, void* workspace, size_t ws_bytes, int32_t splits,
                                      void* stream);
+
+/*
+ * One decode step of the generation path: append each sequence's new token
+ * to the packed cache, then attend over the cache with that step's query.
+ * The pages measure decoding a cache that was packed whole, and name the
+ * complete generation path, appends included, as what a practical claim has
+ * to time ("Block KV decoding: less workspace, more time", section "Use the
+ * failure to choose the next question"); this call is that path.
+ *
+ * Sequence b's new token sits at t = lengths[b] - 1 (lengths count it).  The
+ * call re-packs K group t / g of every (b, h) from the caller's float rows of
+ * that group -- K scales run along tokens, so a group's scale changes as its
+ * tokens arrive -- and packs V row t, in one kernel, then runs kvq_attend with
+ * one query row per sequence.  Afterwards the cache holds, for tokens
+ * [0, lengths[b]), exactly the bytes kvq_pack of those tokens writes.
+ *   Q, cache, H_q, scale, O, workspace, ws_bytes, splits: as kvq_attend with
+ *            Lq = 1 (Q and O [B, H_q, 1, D]; workspace kvq_workspace_size(cache,
+ *            H_q, 1, splits) bytes).
+ *   lengths  device int32 [B]: tokens of each sequence including the new one,
+ *            1..N_cap.
+ *   K_tail   device, [B, H_kv, g, D] in in_dtype: row r of (b, h) holds K of
+ *            token g * (t / g) + r for r = 0 .. t % g (the new token's group
+ *            from its start through the new token); rows after t % g are not
+ *            read (they count as zero, as in a whole-cache pack).
+ *   V_new    device, [B, H_kv, D] in in_dtype: V of the new token.
+ *   in_dtype KVQ_F32 or KVQ_BF16 (bf16 widened exactly to float32 first).
+ * A length outside 1..N_cap is recorded for kvq_check (KVQ_ERR_LENGTH) and
+ * that sequence's cache is left untouched.
+ * Errors: as kvq_attend; KVQ_ERR_ARG (K_tail or V_new NULL, bad in_dtype),
+ * KVQ_ERR_ALIGN (K_tail or V_new not aligned to its element size).
+ */
+KVQ_API kvq_status kvq_decode_step(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                   const int32_t* lengths, const void* K_tail, const void* V_new,
+                                   kvq_dtype in_dtype, int32_t H_q, float scale, void* O, void* workspace,
+                                   size_t ws_bytes, int32_t splits, void* stream);
 
 /*
  * Attention of Q over the packed cache followed by a window of recent tokens
@@ -224,6 +266,32 @@ KVQ_API kvq_status kvq_attend_noalloc(const void* Q, kvq_dtype q_dtype, const kv
 
 /* Size in bytes of the fixed scratch array kvq_attend_noalloc uses. */
 KVQ_API size_t kvq_noalloc_scratch_bytes(void);
+
+/*
+ * Self-test of the bounded waits of the tuned decode kernel (a test hook; the
+ * pages have no counterpart).  Every wait inside the library's kernels is
+ * bounded so that a lost completion ends the kernel with an error instead of
+ * hanging the GPU; this call makes one completion go missing on purpose, on
+ * the host's say-so, without any fault: it runs kvq_attend's decode kernel on
+ * the caller's arguments (Lq = 1; the arguments must select the tuned decode
+ * kernel, else KVQ_ERR_UNSUPPORTED) with every wait limited to wait_ms, and
+ * the first worker's copy of its lose_block-th block arms 16 bytes more than
+ * it brings, so that block's barrier never completes.  That worker's waits
+ * then run out: its pair stops, writes nothing, waits (at most about two
+ * seconds) for the copies it issued, and returns; every other worker
+ * finishes normally.  kvq_check then returns KVQ_ERR_TIMEOUT, within wait_ms
+ * plus about two seconds, and the device stays usable.  The output rows of
+ * the (b, h) pairs that worker covered are not valid.
+ *   lose_block  0-based index of the block in the first worker's range
+ *               (must be one it has; otherwise nothing is lost).
+ *   wait_ms     1..10000.
+ * Errors: as kvq_attend, KVQ_ERR_ARG (lose_block < 0, wait_ms out of range),
+ * KVQ_ERR_UNSUPPORTED.
+ */
+KVQ_API kvq_status kvq_selftest_timeout(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                        const int32_t* lengths, int32_t H_q, float scale, void* O,
+                                        void* workspace, size_t ws_bytes, int32_t splits, int32_t lose_block,
+                                        uint32_t wait_ms, void* stream);
 
 /* Workspace bytes kvq_attend needs for these arguments on the current
  * device (host).  Returns 0 for invalid arguments. */

@@ -12,6 +12,8 @@ is no fallback of any kind.
     O = sm_b200.attend(Q, cache, lengths, scale, causal=True)   # rows = last Lq positions
     O = sm_b200.attend_window(Q, cache, lengths, K_win, V_win, win_lengths, scale)
                                                   # packed tokens, then an unquantized window
+    O = sm_b200.decode_step(Q, cache, lengths, K_tail, V_new, scale)
+                                                  # append each sequence's new token, then attend
 """
 
 from __future__ import annotations
@@ -24,7 +26,7 @@ import torch
 __all__ = [
     "KVQError", "PackedCache", "pack", "attend", "workspace_size", "check",
     "launch_count", "kernel_name", "cache_sizes", "lib", "LIB_PATH", "attend_noalloc",
-    "attend_window", "workspace_size_window",
+    "attend_window", "workspace_size_window", "decode_step",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
@@ -61,6 +63,8 @@ def _load() -> ctypes.CDLL:
     i32, vp, sz = ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
     L.kvq_cache_sizes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]
     L.kvq_cache_sizes.restype = ctypes.c_int
+    L.kvq_cache_bytes.argtypes = [ctypes.POINTER(_Cache)]
+    L.kvq_cache_bytes.restype = sz
     L.kvq_pack.argtypes = [vp, vp, ctypes.c_int, i32, i32, ctypes.POINTER(_Cache), vp]
     L.kvq_pack.restype = ctypes.c_int
     L.kvq_attend.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, i32, i32,
@@ -89,6 +93,12 @@ def _load() -> ctypes.CDLL:
     L.kvq_attend_window.restype = ctypes.c_int
     L.kvq_workspace_size_window.argtypes = [ctypes.POINTER(_Cache), i32, i32, i32]
     L.kvq_workspace_size_window.restype = sz
+    L.kvq_decode_step.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, vp, vp, ctypes.c_int, i32,
+                                  ctypes.c_float, vp, vp, sz, i32, vp]
+    L.kvq_decode_step.restype = ctypes.c_int
+    L.kvq_selftest_timeout.argtypes = [vp, ctypes.c_int, ctypes.POINTER(_Cache), vp, i32, ctypes.c_float, vp, vp,
+                                       sz, i32, i32, ctypes.c_uint32, vp]
+    L.kvq_selftest_timeout.restype = ctypes.c_int
     return L
 
 
@@ -153,8 +163,7 @@ class PackedCache:
         return -(-self.D // self.group) * self.group
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in
-                   (self.k_codes, self.k_scales, self.v_codes, self.v_scales))
+        return int(lib.kvq_cache_bytes(ctypes.byref(self._struct)))
 
     def struct(self) -> _Cache:
         return self._struct
@@ -275,6 +284,47 @@ def attend_noalloc(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, s
     _ok(lib.kvq_attend_noalloc(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(),
                                int(Q.shape[1]), int(Q.shape[2]), float(scale), out.data_ptr(),
                                int(splits), _stream(cache.device)), "kvq_attend_noalloc")
+    return out
+
+
+def decode_step(Q: torch.Tensor, cache: PackedCache, lengths: torch.Tensor, K_tail: torch.Tensor,
+                V_new: torch.Tensor, scale: float, out: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, splits: int = 0) -> torch.Tensor:
+    """One decode step: append each sequence's new token (position
+    lengths[b] - 1) to the packed cache and attend over it.  K_tail
+    [B, H_kv, g, D] holds the K rows of each sequence's last group from its
+    start through the new token (later rows are not read); V_new
+    [B, H_kv, D] (or [B, H_kv, 1, D]) the new token's V.  Q [B, H_q, 1, D];
+    lengths int32 [B] on the device, counting the new token.  Returns O like Q."""
+    _check_cuda(Q, "Q", cache.device)
+    _check_cuda(lengths, "lengths", cache.device)
+    if lengths.dtype != torch.int32 or lengths.numel() != cache.B:
+        raise ValueError("lengths must be int32 [B]")
+    if Q.dim() != 4 or Q.shape[0] != cache.B or Q.shape[2] != 1 or Q.shape[3] != cache.D:
+        raise ValueError("Q must be [B, H_q, 1, D]")
+    _check_cuda(K_tail, "K_tail", cache.device)
+    _check_cuda(V_new, "V_new", cache.device)
+    if tuple(K_tail.shape) != (cache.B, cache.H_kv, cache.group, cache.D):
+        raise ValueError("K_tail must be [B, H_kv, group, D]")
+    if V_new.numel() != cache.B * cache.H_kv * cache.D or V_new.shape[0] != cache.B:
+        raise ValueError("V_new must be [B, H_kv, D]")
+    if K_tail.dtype != V_new.dtype:
+        raise ValueError("K_tail and V_new must have one dtype")
+    H_q = int(Q.shape[1])
+    if out is None:
+        out = torch.empty_like(Q)
+    else:
+        _check_cuda(out, "out", cache.device)
+        if out.shape != Q.shape or out.dtype != Q.dtype:
+            raise ValueError("out must match Q")
+    need = workspace_size(cache, H_q, 1, splits)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=cache.device)
+    c = cache.struct()
+    _ok(lib.kvq_decode_step(Q.data_ptr(), _dtype_code(Q), ctypes.byref(c), lengths.data_ptr(),
+                            K_tail.data_ptr(), V_new.data_ptr(), _dtype_code(K_tail), H_q, float(scale),
+                            out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            int(splits), _stream(cache.device)), "kvq_decode_step")
     return out
 
 

@@ -663,7 +663,7 @@ int rows_per_head(const AttendArgs& a) { return (a.H_q / a.g.H_kv) * a.Lq; }
 bool chunk_applies(const AttendArgs& a) {
   const int R = rows_per_head(a);
   return a.g.D == kD && a.g.group == 32 && (a.g.bits == 4 || a.g.bits == 8) && a.q_dtype == KVQ_BF16 &&
-         (R == 128 || R == 256) && (reinterpret_cast<uintptr_t>(a.Q) & 15u) == 0 &&
+         (R == 128 || R == 256) &&
          static_cast<long long>(a.g.B) * a.H_q * a.Lq < (1LL << 31) && smem_bytes(a.g.B) <= 227 * 1024;
 }
 

@@ -148,6 +148,14 @@ kvq_status kvq_cache_sizes(int32_t bits, int32_t group, int32_t B, int32_t H_kv,
   return KVQ_OK;
 }
 
+size_t kvq_cache_bytes(const kvq_cache* cache) {
+  if (!cache) return 0;
+  size_t sizes[4];
+  if (kvq_cache_sizes(cache->bits, cache->group, cache->B, cache->H_kv, cache->N_cap, cache->D, sizes) != KVQ_OK)
+    return 0;
+  return sizes[0] + sizes[1] + sizes[2] + sizes[3];
+}
+
 kvq_status kvq_pack(const void* K, const void* V, kvq_dtype in_dtype, int32_t t0, int32_t t1,
                     const kvq_cache* cache, void* stream) {
   PackArgs a{};
@@ -182,14 +190,16 @@ size_t kvq_workspace_size(const kvq_cache* cache, int32_t H_q, int32_t Lq, int32
   return impl.workspace(a);
 }
 
-static kvq_status attend_common(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
-                                const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
-                                void* workspace, size_t ws_bytes, int32_t splits, bool causal, void* stream) {
-  AttendArgs a{};
+// Every argument rule of the attend calls, checked on the host before any
+// launch; on success *impl is the implementation that will run.
+static kvq_status attend_prepare(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                 const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
+                                 void* workspace, size_t ws_bytes, int32_t splits, bool causal, AttendArgs* a,
+                                 const AttendImpl** impl) {
   if (!fill_attend_args(Q, q_dtype, cache, lengths, H_q, Lq, scale, O, workspace, ws_bytes,
-                        splits, &a))
+                        splits, a))
     return KVQ_ERR_ARG;
-  a.causal = causal && Lq > 1;             // one query row at the last position sees every key
+  a->causal = causal && Lq > 1;            // one query row at the last position sees every key
   if (!Q || !O || !lengths || !cache->k_codes || !cache->k_scales || !cache->v_codes ||
       !cache->v_scales)
     return KVQ_ERR_ARG;
@@ -198,16 +208,28 @@ static kvq_status attend_common(const void* Q, kvq_dtype q_dtype, const kvq_cach
   if (!aligned16(cache->k_codes) || !aligned16(cache->k_scales) || !aligned16(cache->v_codes) ||
       !aligned16(cache->v_scales))
     return KVQ_ERR_ALIGN;
-  const size_t esz = q_dtype == KVQ_F32 ? 4 : 2;
-  if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) % esz) return KVQ_ERR_ALIGN;
+  // Q and O 16-byte aligned whatever their dtype, so that the kernel chosen
+  // (and the workspace kvq_workspace_size reported) never depends on an address
+  if (!aligned16(Q) || !aligned16(O)) return KVQ_ERR_ALIGN;
   if (reinterpret_cast<uintptr_t>(lengths) % 4) return KVQ_ERR_ALIGN;
-  const AttendImpl& impl = choose(a);
-  const size_t need = impl.workspace(a);
+  *impl = &choose(*a);
+  const size_t need = (*impl)->workspace(*a);
   if (need > 0) {
     if (!workspace || ws_bytes < need) return KVQ_ERR_WORKSPACE;
     if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
   }
-  return impl.launch(a, static_cast<cudaStream_t>(stream));
+  return KVQ_OK;
+}
+
+static kvq_status attend_common(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                const int32_t* lengths, int32_t H_q, int32_t Lq, float scale, void* O,
+                                void* workspace, size_t ws_bytes, int32_t splits, bool causal, void* stream) {
+  AttendArgs a{};
+  const AttendImpl* impl = nullptr;
+  const kvq_status st = attend_prepare(Q, q_dtype, cache, lengths, H_q, Lq, scale, O, workspace, ws_bytes,
+                                       splits, causal, &a, &impl);
+  if (st != KVQ_OK) return st;
+  return impl->launch(a, static_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_attend(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
@@ -222,6 +244,50 @@ kvq_status kvq_attend_causal(const void* Q, kvq_dtype q_dtype, const kvq_cache* 
                              void* workspace, size_t ws_bytes, int32_t splits, void* stream) {
   return attend_common(Q, q_dtype, cache, lengths, H_q, Lq, scale, O, workspace, ws_bytes, splits, true,
                        stream);
+}
+
+kvq_status kvq_decode_step(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                           const int32_t* lengths, const void* K_tail, const void* V_new, kvq_dtype in_dtype,
+                           int32_t H_q, float scale, void* O, void* workspace, size_t ws_bytes, int32_t splits,
+                           void* stream) {
+  AttendArgs a{};
+  const AttendImpl* impl = nullptr;
+  const kvq_status st = attend_prepare(Q, q_dtype, cache, lengths, H_q, 1, scale, O, workspace, ws_bytes,
+                                       splits, false, &a, &impl);
+  if (st != KVQ_OK) return st;
+  if (!K_tail || !V_new || (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16)) return KVQ_ERR_ARG;
+  const size_t esz = in_dtype == KVQ_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(K_tail) | reinterpret_cast<uintptr_t>(V_new)) % esz) return KVQ_ERR_ALIGN;
+  AppendArgs ap{};
+  ap.K_tail = K_tail;
+  ap.V_new = V_new;
+  ap.in_dtype = in_dtype;
+  ap.lengths = lengths;
+  ap.g = a.g;
+  ap.k_codes = cache->k_codes;
+  ap.k_scales = cache->k_scales;
+  ap.v_codes = cache->v_codes;
+  ap.v_scales = cache->v_scales;
+  if (append_smem_bytes(a.g) > 227 * 1024 || a.g.H_kv > 65535) return KVQ_ERR_UNSUPPORTED;
+  const kvq_status ast = launch_append(ap, static_cast<cudaStream_t>(stream));
+  if (ast != KVQ_OK) return ast;
+  return impl->launch(a, static_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_selftest_timeout(const void* Q, kvq_dtype q_dtype, const kvq_cache* cache,
+                                const int32_t* lengths, int32_t H_q, float scale, void* O, void* workspace,
+                                size_t ws_bytes, int32_t splits, int32_t lose_block, uint32_t wait_ms,
+                                void* stream) {
+  AttendArgs a{};
+  const AttendImpl* impl = nullptr;
+  const kvq_status st = attend_prepare(Q, q_dtype, cache, lengths, H_q, 1, scale, O, workspace, ws_bytes,
+                                       splits, false, &a, &impl);
+  if (st != KVQ_OK) return st;
+  if (impl != decode_attend_impl()) return KVQ_ERR_UNSUPPORTED;
+  if (lose_block < 0 || wait_ms < 1 || wait_ms > 10000) return KVQ_ERR_ARG;
+  a.test_lose_block = lose_block;
+  a.test_wait_ns = static_cast<unsigned long long>(wait_ms) * 1000000ull;
+  return impl->launch(a, static_cast<cudaStream_t>(stream));
 }
 
 static bool fill_window(const void* K_win, const void* V_win, kvq_dtype win_dtype,
@@ -266,8 +332,7 @@ kvq_status kvq_attend_window(const void* Q, kvq_dtype q_dtype, const kvq_cache* 
   if (!aligned16(cache->k_codes) || !aligned16(cache->k_scales) || !aligned16(cache->v_codes) ||
       !aligned16(cache->v_scales))
     return KVQ_ERR_ALIGN;
-  const size_t esz = q_dtype == KVQ_F32 ? 4 : 2;
-  if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(O)) % esz) return KVQ_ERR_ALIGN;
+  if (!aligned16(Q) || !aligned16(O)) return KVQ_ERR_ALIGN;
   const size_t wsz = win_dtype == KVQ_F32 ? 4 : 2;
   if ((reinterpret_cast<uintptr_t>(K_win) | reinterpret_cast<uintptr_t>(V_win)) % wsz) return KVQ_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(lengths) | reinterpret_cast<uintptr_t>(win_lengths)) % 4) return KVQ_ERR_ALIGN;

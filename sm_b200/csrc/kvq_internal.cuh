@@ -172,6 +172,22 @@ struct PackArgs {
 };
 kvq_status launch_pack(const PackArgs& a, cudaStream_t s);
 
+// Decode-step append (kvq_decode_step): re-pack the K group holding each
+// sequence's new token t = lengths[b] - 1 from its float rows, pack V row t.
+struct AppendArgs {
+  const void* K_tail;              // [B, H_kv, g, D]
+  const void* V_new;               // [B, H_kv, D]
+  int in_dtype;
+  const int32_t* lengths;
+  Geometry g;
+  uint8_t* k_codes;
+  float* k_scales;
+  uint8_t* v_codes;
+  float* v_scales;
+};
+size_t append_smem_bytes(const Geometry& g);
+kvq_status launch_append(const AppendArgs& a, cudaStream_t s);
+
 struct AttendArgs {
   const void* Q;
   int q_dtype;
@@ -194,6 +210,11 @@ struct AttendArgs {
   int win_dtype;
   const int32_t* win_lengths;
   int W_cap;
+  // self-test of the tuned decode kernel's timeout path (kvq_selftest_timeout):
+  // worker 0 loses the completion of its test_lose_block-th block and every
+  // wait is bounded by test_wait_ns; -1 / 0: none, the default limit
+  int test_lose_block = -1;
+  unsigned long long test_wait_ns = 0;
 };
 
 // Workspace of an implementation whose packed partials fill `slots` slots of

@@ -205,7 +205,153 @@ __global__ void __launch_bounds__(256) pack_v128_kernel(PackParams p) {
   }
 }
 
+// Decode-step append: one CTA per (h, b).  Sequence b's new token sits at
+// t = lengths[b] - 1.  The CTA re-packs K group t / g from the caller's
+// float rows of that group (rows past t % g read as zero, as a whole-cache
+// pack pads a short last group) and packs V row t; what it writes is exactly
+// what kvq_pack of tokens [0, lengths[b]) writes for that group and row.
+struct AppendParams {
+  const void* K_tail;        // [B, H, g, D]
+  const void* V_new;         // [B, H, D]
+  int dtype;
+  const int32_t* lengths;
+  int bits, group, B, H, D, Dp, N_cap;
+  long long k_codes_head, k_scales_head, v_codes_head, v_scales_head;
+  uint8_t* k_codes;
+  float* k_scales;
+  uint8_t* v_codes;
+  float* v_scales;
+  unsigned int* err;
+};
+
+__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+  griddep_wait();
+  extern __shared__ float s_x[];                   // [g][D] tail rows, then scale[D], 1/scale[D]
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int L = p.lengths[b];
+  if (L < 1 || L > p.N_cap) {
+    if (threadIdx.x == 0 && h == 0) record_error(p.err, KVQ_ERR_LENGTH);
+    return;
+  }
+  const int g = p.group, D = p.D;
+  const int qmax = p.bits == 4 ? 7 : 127;
+  const int t = L - 1, j = t / g, nin = t % g + 1;
+  const long long head = static_cast<long long>(b) * p.H + h;
+
+  // K: the group's rows into shared memory, loads issued in batches
+  const int n = g * D;
+  const long long kin = head * n;
+  constexpr int U = 8;
+  for (int i0 = 0; i0 < n; i0 += U * static_cast<int>(blockDim.x)) {
+    float v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * static_cast<int>(blockDim.x) + threadIdx.x;
+      v[u] = (i < n && i / D < nin) ? load_as_f32(p.K_tail, kin + i, p.dtype) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * static_cast<int>(blockDim.x) + threadIdx.x;
+      if (i < n) s_x[i] = v[u];
+    }
+  }
+  __syncthreads();
+  float* s_scale = s_x + n;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float amax = 0.f;
+    for (int tt = 0; tt < nin; ++tt) amax = fmaxf(amax, fabsf(s_x[tt * D + d]));
+    const float sc = group_scale(amax, qmax);
+    s_scale[d] = sc;
+    s_scale[D + d] = __frcp_rn(sc);
+    p.k_scales[head * p.k_scales_head + static_cast<long long>(j) * D + d] = sc;
+  }
+  __syncthreads();
+  const long long code0 = static_cast<long long>(j) * n;           // flat index of the group start
+  uint8_t* kout = p.k_codes + head * p.k_codes_head;
+  if (p.bits == 4) {
+    for (int jb = threadIdx.x; jb < n / 2; jb += blockDim.x) {
+      const int f = 2 * jb;
+      const int d0 = f % D, d1 = (f + 1) % D;
+      const unsigned lo = quant_code(s_x[f], s_scale[d0], s_scale[D + d0], qmax);
+      const unsigned hi = quant_code(s_x[f + 1], s_scale[d1], s_scale[D + d1], qmax);
+      kout[code0 / 2 + jb] = static_cast<uint8_t>(lo | (hi << 4));
+    }
+  } else {
+    for (int f = threadIdx.x; f < n; f += blockDim.x)
+      kout[code0 + f] = static_cast<uint8_t>(quant_code(s_x[f], s_scale[f % D], s_scale[D + f % D], qmax));
+  }
+
+  // V row t: warp w takes feature groups w, w + warps, ...; features past D
+  // are the zero padding of the last group
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int ng = p.Dp / g;
+  const long long vin = head * D;
+  uint8_t* vout = p.v_codes + head * p.v_codes_head;
+  for (int gj = warp; gj < ng; gj += nw) {
+    const int d0 = gj * g;
+    float amax = 0.f;
+    for (int e = lane; e < g; e += 32)
+      if (d0 + e < D) amax = fmaxf(amax, fabsf(load_as_f32(p.V_new, vin + d0 + e, p.dtype)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = group_scale(amax, qmax);
+    const float rs = __frcp_rn(sc);
+    if (lane == 0) p.v_scales[head * p.v_scales_head + static_cast<long long>(t) * ng + gj] = sc;
+    const long long c0 = static_cast<long long>(t) * p.Dp + d0;     // even: Dp and d0 are multiples of g
+    if (p.bits == 4) {
+      for (int e = 2 * lane; e < g; e += 64) {
+        const float x0 = d0 + e < D ? load_as_f32(p.V_new, vin + d0 + e, p.dtype) : 0.f;
+        const float x1 = d0 + e + 1 < D ? load_as_f32(p.V_new, vin + d0 + e + 1, p.dtype) : 0.f;
+        vout[(c0 + e) / 2] = static_cast<uint8_t>(quant_code(x0, sc, rs, qmax) | (quant_code(x1, sc, rs, qmax) << 4));
+      }
+    } else {
+      for (int e = lane; e < g; e += 32) {
+        const float x = d0 + e < D ? load_as_f32(p.V_new, vin + d0 + e, p.dtype) : 0.f;
+        vout[c0 + e] = static_cast<uint8_t>(quant_code(x, sc, rs, qmax));
+      }
+    }
+  }
+}
+
 }  // namespace
+
+size_t append_smem_bytes(const Geometry& g) {
+  return (static_cast<size_t>(g.group) * g.D + 2 * static_cast<size_t>(g.D)) * sizeof(float);
+}
+
+kvq_status launch_append(const AppendArgs& a, cudaStream_t s) {
+  const Geometry& g = a.g;
+  if (g.B > 65535 || g.H_kv > 65535) return KVQ_ERR_UNSUPPORTED;
+  const size_t smem = append_smem_bytes(g);
+  if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
+  if (smem > 48 * 1024 && !ensure_dynamic_smem(reinterpret_cast<const void*>(append_kernel), smem))
+    return KVQ_ERR_CUDA;
+  AppendParams p{};
+  p.K_tail = a.K_tail;
+  p.V_new = a.V_new;
+  p.dtype = a.in_dtype;
+  p.lengths = a.lengths;
+  p.bits = g.bits;
+  p.group = g.group;
+  p.B = g.B;
+  p.H = g.H_kv;
+  p.D = g.D;
+  p.Dp = g.Dp;
+  p.N_cap = g.N_cap;
+  p.k_codes_head = static_cast<long long>(g.k_codes_head);
+  p.k_scales_head = static_cast<long long>(g.k_scales_head);
+  p.v_codes_head = static_cast<long long>(g.v_codes_head);
+  p.v_scales_head = static_cast<long long>(g.v_scales_head);
+  p.k_codes = a.k_codes;
+  p.k_scales = a.k_scales;
+  p.v_codes = a.v_codes;
+  p.v_scales = a.v_scales;
+  p.err = error_word();
+  if (!p.err) return KVQ_ERR_CUDA;
+  if (launch_pdl(append_kernel, dim3(g.H_kv, g.B), dim3(256), smem, s, p) != cudaSuccess) return KVQ_ERR_CUDA;
+  count_launch();
+  return KVQ_OK;
+}
 
 kvq_status launch_pack(const PackArgs& a, cudaStream_t s) {
   const Geometry& g = a.g;

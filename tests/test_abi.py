@@ -104,11 +104,29 @@ def test_attend_argument_rules():
     assert call(q=0) == 1 and call(o=0) == 1 and call(lens=0) == 1
     assert call(cache=_cache(ptr=0x10008)) == 3  # cache arrays not 16-byte aligned
     assert call(q=0x1001) == 3                   # bf16 Q misaligned
+    # Q and O must be 16-byte aligned whatever their dtype: a bf16 Q two bytes
+    # off would otherwise change which kernel runs after kvq_workspace_size
+    # sized the workspace for another
+    assert call(q=0x1002) == 3
+    assert call(q=0x1008, dt=K.KVQ_F32) == 3
+    assert call(o=0x4002) == 3
     assert call(lens=0x3002) == 3
     assert call(cache=_cache(D=300)) == 8        # unsupported width
     assert call(w=0) == 4                        # no workspace
     assert call(wsb=16) == 4                     # too small
     assert call(w=0x5008) == 3                   # misaligned workspace
+
+
+def test_cache_bytes_is_the_sum_of_the_array_sizes():
+    for shape in [(4, 32, 3, 2, 128, 32), (4, 8, 1, 1, 35, 13), (8, 32, 32, 8, 4096, 128)]:
+        bits, group, B, H, N, D = shape
+        c = K._Cache(bits, group, B, H, N, D, 0, 0, 0, 0)
+        assert K.lib.kvq_cache_bytes(ctypes.byref(c)) == sum(K.cache_sizes(B, H, N, D, bits, group))
+    assert K.lib.kvq_cache_bytes(ctypes.byref(_cache(bits=5))) == 0
+    assert K.lib.kvq_cache_bytes(None) == 0
+    # the decode workload's cache: 168 MB, as the byte accounting says
+    c = K._Cache(4, 32, 32, 8, 4096, 128, 0, 0, 0, 0)
+    assert K.lib.kvq_cache_bytes(ctypes.byref(c)) == 32 * 8 * (4096 * 64 * 2 + 128 * 128 * 4 + 4096 * 4 * 4)
 
 
 def test_workspace_size_grows_with_splits():
@@ -157,3 +175,42 @@ def test_causal_argument_rules():
     assert call(lens=0x3002) == 3
     assert call(w=0) == 4
     assert call(wsb=16) == 4
+
+
+def test_decode_step_argument_rules():
+    """kvq_decode_step takes kvq_attend's rules with Lq = 1, plus its two
+    input rows; every call here fails on the host before any launch."""
+    c = _cache()
+
+    def call(q=0x1000, lens=0x3000, kt=0x6000, vn=0x7000, dt=K.KVQ_F32, hq=4, w=0x5000, wsb=1 << 30, o=0x4000):
+        return K.lib.kvq_decode_step(q, K.KVQ_BF16, ctypes.byref(c), lens, kt, vn, dt, hq, 1.0, o, w, wsb, 0,
+                                     None)
+
+    assert call(hq=3) == 1
+    assert call(kt=0) == 1 and call(vn=0) == 1
+    assert call(dt=5) == 1
+    assert call(kt=0x6002) == 3                 # float32 rows misaligned
+    assert call(vn=0x7001, dt=K.KVQ_BF16) == 3
+    assert call(q=0x1002) == 3 and call(o=0x4008) == 3
+    assert call(lens=0x3002) == 3
+    assert call(w=0) == 4
+    assert call(wsb=16) == 4
+    assert K.lib.kvq_decode_step(0x1000, K.KVQ_BF16, ctypes.byref(_cache(bits=3)), 0x3000, 0x6000, 0x7000,
+                                 K.KVQ_F32, 4, 1.0, 0x4000, 0x5000, 1 << 30, 0, None) == 1
+
+
+def test_selftest_argument_rules_host():
+    """kvq_selftest_timeout checks its arguments on the host (no launch)."""
+    c = _cache(B=2, H=2, N=512, D=128)
+
+    def call(lb=1, ms=100, hq=8, w=0x5000, wsb=1 << 30):
+        return K.lib.kvq_selftest_timeout(0x1000, K.KVQ_BF16, ctypes.byref(c), 0x3000, hq, 1.0, 0x4000, w, wsb, 0,
+                                          lb, ms, None)
+
+    assert call(lb=-1) == 1
+    assert call(ms=0) == 1 and call(ms=10001) == 1
+    assert call(hq=3) == 1
+    assert call(w=0) == 4
+    c64 = _cache(B=2, H=2, N=512, D=64)            # not the tuned decode kernel
+    assert K.lib.kvq_selftest_timeout(0x1000, K.KVQ_BF16, ctypes.byref(c64), 0x3000, 8, 1.0, 0x4000, 0x5000,
+                                      1 << 30, 0, 1, 100, None) == 8
