@@ -88,6 +88,7 @@ struct Tr {
   static constexpr float kCorrOdd = BITS == 4 ? 1.f + 7.f / 16.f : 1.f + 127.f / 256.f;
 };
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazy = 8.f;          // rescale threshold of the running reference, log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int BITS, int GRP>
@@ -113,6 +114,8 @@ struct PairSmem {
   unsigned long long cursor[2][6];    // each warp's copy cursor (a Prod), lane 0's alone
   unsigned long long pfull[2];        // S-warp wrote part[i]
   unsigned long long pempty[2];       // V-warp read part[i]
+  int abort;                          // a wait of this pair ran out: both warps stop
+  int pad_[3];
 };
 
 static_assert(sizeof(Stage<4, 32>) % 16 == 0 && sizeof(Stage<8, 32>) % 16 == 0 &&
@@ -138,6 +141,10 @@ struct DecodeParams {
   int ctas;                           // CTAs; each warp pair is one worker of the plan
   int force_partial;                  // a window follows: no worker writes output rows
   unsigned int* err;
+  unsigned long long wait_ns;         // limit of every bounded wait
+  int lose_worker, lose_block;        // self-test of the timeout path: this worker's K copy of its
+                                      // lose_block-th block arms 16 bytes more than it brings, so
+                                      // that block's barrier never completes; -1: none
 };
 
 // shared memory after the pairs: pre [B + 1], len [B]
@@ -210,18 +217,43 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// Bounded wait: gives up after about two seconds, records KVQ_ERR_TIMEOUT and
-// returns false, so a lost completion ends the kernel instead of hanging it.
-__device__ __forceinline__ bool wait_bar(unsigned long long* bar, uint32_t parity,
-                                         unsigned int* err) {
+// Bounded wait of one warp on a phase of `bar`.  Returns true once the phase
+// completed.  Returns false when the pair's abort flag is up (the other warp
+// gave up), or after limit_ns: then it raises the flag itself and records
+// KVQ_ERR_TIMEOUT.  So one lost completion ends the pair's work within one
+// limit, and every later wait of the pair returns at once.
+__device__ __forceinline__ bool wait_bar(unsigned long long* bar, uint32_t parity, unsigned int* err,
+                                         volatile int* abort, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
+  bool ok = false;
+  if (!*abort) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try_wait_sleep(bar, parity)) {
+        ok = true;
+        break;
+      }
+      if ((it & 7u) == 0) {
+        if (*abort) break;
+        if (globaltimer() - t0 > limit_ns) {
+          *abort = 1;
+          record_error(err, KVQ_ERR_TIMEOUT);
+          break;
+        }
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+// After an abort: wait (at most about two seconds) for a bulk copy this warp
+// issued into `bar` to land, so no copy is still writing shared memory when
+// the CTA exits.
+__device__ __forceinline__ void drain_bar(unsigned long long* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
-    if ((it & 7u) == 0 && globaltimer() - t0 > 2000000000ull) {
-      record_error(err, KVQ_ERR_TIMEOUT);
-      return false;
-    }
+    if (mbar_try_wait_sleep(bar, parity)) return;
+    if ((it & 7u) == 0 && globaltimer() - t0 > 2000000000ull) return;
   }
 }
 
@@ -278,6 +310,64 @@ __device__ __forceinline__ void code_pairs(const uint8_t* codes, int t, int cs, 
   } else {
     const uint4 w = *reinterpret_cast<const uint4*>(codes + t * 128 + cs * 16);
     byte_pairs15(w, f);
+  }
+}
+
+// V codes as exact offsets (code - qmax) * eps with one shift per four
+// bytes.  The offset is taken per pair as f - (1 + qmax eps), which is exact
+// for any eps (both terms lie in [1, 2)), so V needs no cancellation-safe
+// placement: a code may sit anywhere its mantissa field stays below the
+// exponent.  Per 32-bit word w (channels in byte order) and v = w >> 16, the
+// channels keep their order: 4-bit pairs (ch 0, ch 1) and (ch 4, ch 5) at
+// eps (2^-23, 2^-19), from w and v; (ch 2, ch 3) and (ch 6, ch 7) at
+// (2^-15, 2^-11).  8-bit pairs (ch 0, ch 1) and (ch 2, ch 3) at
+// (2^-23, 2^-15).  So two correction pairs at 4 bits and one at 8.
+template <int BITS>
+struct VSlot {
+  // 1/eps of half j of pair i, at [2i + j]
+  static constexpr float inv_eps(int k) {
+    return BITS == 4 ? ((k & 3) == 0 ? 8388608.f : (k & 3) == 1 ? 524288.f : (k & 3) == 2 ? 32768.f : 2048.f)
+                     : ((k & 1) == 0 ? 8388608.f : 32768.f);
+  }
+};
+
+__device__ __forceinline__ uint32_t mant_or(uint32_t x, uint32_t mask) {
+  uint32_t y;
+  asm("lop3.b32 %0, %1, %2, 0x3F800000, 0xEA;" : "=r"(y) : "r"(x), "r"(mask));
+  return y;
+}
+
+__device__ __forceinline__ u64 pair_u32(uint32_t lo, uint32_t hi) {
+  u64 v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+  return v;
+}
+
+// 1 + qmax * 2^(p - 23)
+constexpr float vcorr(int qmax, int p) { return 1.f + static_cast<float>(qmax) / static_cast<float>(1 << (23 - p)); }
+
+// The lane's 16 V channels of token t as eight exact offset pairs, channel
+// 2i and 2i + 1 in pair i.
+template <int BITS>
+__device__ __forceinline__ void v_offsets(const uint8_t* codes, int t, int cs, u64 f[8]) {
+  if (BITS == 4) {
+    const uint2 w2 = *reinterpret_cast<const uint2*>(codes + t * 64 + cs * 8);
+    const u64 c01 = pack2(-vcorr(7, 0), -vcorr(7, 4)), c23 = pack2(-vcorr(7, 8), -vcorr(7, 12));
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const uint32_t w = (h < 2 ? w2.x : w2.y) >> (16 * (h & 1));
+      f[2 * h] = add2(pair_u32(mant_or(w, 0x000Fu), mant_or(w, 0x00F0u)), c01);
+      f[2 * h + 1] = add2(pair_u32(mant_or(w, 0x0F00u), mant_or(w, 0xF000u)), c23);
+    }
+  } else {
+    const uint4 w4 = *reinterpret_cast<const uint4*>(codes + t * 128 + cs * 16);
+    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+    const u64 c = pack2(-vcorr(127, 0), -vcorr(127, 8));
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const uint32_t w = ws[h >> 1] >> (16 * (h & 1));
+      f[h] = add2(pair_u32(mant_or(w, 0x00FFu), mant_or(w, 0xFF00u)), c);
+    }
   }
 }
 
@@ -363,7 +453,7 @@ __device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H
 // block's groups holding valid tokens, and the V scales.
 template <int BITS, int GRP>
 __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS, GRP>& ps, int stage, int b,
-                                            int h, int j, const int* slen) {
+                                            int h, int j, const int* slen, uint32_t extra) {
   const long long head = static_cast<long long>(b) * p.H + h;
   const int len = slen[b];
   const int t0 = j * kTB;
@@ -373,7 +463,7 @@ __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS
   unsigned long long* bar = &ps.full[stage];
   constexpr int kVs = Tr<BITS, GRP>::kVs;
   const int krows = (nv + GRP - 1) / GRP;                // K groups holding valid tokens
-  mbar_expect_tx(bar, static_cast<uint32_t>((2 * kCb + kVs * 4) * nv + krows * kD * 4));
+  mbar_expect_tx(bar, static_cast<uint32_t>((2 * kCb + kVs * 4) * nv + krows * kD * 4) + extra);
   bulk_g2s(st.kc, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
   bulk_g2s(st.vc, p.v_codes + head * p.v_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
   bulk_g2s(st.ks, p.k_scales + head * p.k_scales_head + static_cast<long long>(t0 / GRP) * kD,
@@ -389,7 +479,7 @@ __device__ __forceinline__ void issue_block(const DecodeParams& p, PairSmem<BITS
 // the half's barrier with its byte count and issues its two copies.
 template <int BITS, int GRP>
 __device__ __forceinline__ void issue_half(const DecodeParams& p, PairSmem<BITS, GRP>& ps, int stage, int b,
-                                           int h, int j, const int* slen, bool k_half) {
+                                           int h, int j, const int* slen, bool k_half, uint32_t extra) {
   const long long head = static_cast<long long>(b) * p.H + h;
   const int len = slen[b];
   const int t0 = j * kTB;
@@ -400,7 +490,7 @@ __device__ __forceinline__ void issue_half(const DecodeParams& p, PairSmem<BITS,
   if (k_half) {
     unsigned long long* bar = &ps.full[stage];
     const int krows = (nv + GRP - 1) / GRP;                // K groups holding valid tokens
-    mbar_expect_tx(bar, static_cast<uint32_t>(kCb * nv + krows * kD * 4));
+    mbar_expect_tx(bar, static_cast<uint32_t>(kCb * nv + krows * kD * 4) + extra);
     bulk_g2s(st.kc, p.k_codes + head * p.k_codes_head + static_cast<long long>(t0) * kCb, nv * kCb, bar);
     bulk_g2s(st.ks, p.k_scales + head * p.k_scales_head + static_cast<long long>(t0 / GRP) * kD,
              krows * kD * sizeof(float), bar);
@@ -445,6 +535,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       mbar_init(&ps.pfull[i], 1);
       mbar_init(&ps.pempty[i], 1);
     }
+    ps.abort = 0;
   }
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
@@ -486,12 +577,22 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       ps.qs[qs_index(i / kD, i % kD)] = qv[r] * qf;
     }
   };
+  // Copies this warp issued (whole refill: the S-warp's blocks; split: each
+  // warp's halves, counted by lane 0) and the waits on them that completed:
+  // after an abort the difference is drained before the CTA exits.
+  uint32_t issued = 0, landed = 0;
+  // the self-test's lost completion: 16 bytes armed that no copy brings
+  auto extra_tx = [&](bool k_half) -> uint32_t {
+    return (k_half && worker == p.lose_worker && issued == static_cast<uint32_t>(p.lose_block)) ? 16u : 0u;
+  };
+  volatile int* abort = &ps.abort;
   if (is_s) load_q(seg);
   if constexpr (kSplit) {
     if (lane == 0) {
       Prod pr = prod;
       for (int s = 0; s < kS && pr.valid; ++s) {
-        issue_half<BITS, GRP>(p, ps, s, pr.seg.b, pr.seg.h, pr.j, slen, is_s);
+        issue_half<BITS, GRP>(p, ps, s, pr.seg.b, pr.seg.h, pr.j, slen, is_s, extra_tx(is_s));
+        ++issued;
         ++pr.j;
         pr = prod_settle(pr, pre, p.B, H, cr);
       }
@@ -499,7 +600,8 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
     }
   } else if (is_s) {
     for (int s = 0; s < kS && prod.valid; ++s) {
-      if (lane == 0) issue_block<BITS, GRP>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen);
+      if (lane == 0) issue_block<BITS, GRP>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen, extra_tx(true));
+      ++issued;
       ++prod.j;
       prod = prod_settle(prod, pre, p.B, H, cr);
     }
@@ -508,7 +610,8 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
 
   uint32_t k = 0;                                        // blocks this pair has consumed
   bool first = true;
-  while (seg.valid) {
+  bool alive = true;                                     // no wait of the pair ran out
+  while (seg.valid && alive) {
     const int b = seg.b, h = seg.h;
     const long long head = static_cast<long long>(b) * H + h;
     const long long qrow = static_cast<long long>(b) * H * kG + static_cast<long long>(h) * kG;
@@ -526,7 +629,11 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
-        wait_bar(&ps.full[stage], (k / kS) & 1u, p.err);
+        if (!wait_bar(&ps.full[stage], (k / kS) & 1u, p.err, abort, p.wait_ns)) {
+          alive = false;
+          break;
+        }
+        ++landed;
         const Stage& st = ps.st[stage];
 
         // q'' = q * scale * log2e / eps * s_k, as channel pairs (16cs + 2i, +1)
@@ -556,7 +663,10 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
           }
         }
         // the V-warp must have read this partial buffer's previous block
-        if (k >= 2) wait_bar(&ps.pempty[pb], ((k - 2) >> 1) & 1u, p.err);
+        if (k >= 2 && !wait_bar(&ps.pempty[pb], ((k - 2) >> 1) & 1u, p.err, abort, p.wait_ns)) {
+          alive = false;
+          break;
+        }
         float* part = ps.part[pb];
 #pragma unroll 2
         for (int it = 0; it < kTB / 4; ++it) {
@@ -584,7 +694,8 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
             Prod pr = *cur;
             if (pr.valid) {
               fence_proxy_async();
-              issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, true);
+              issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, true, extra_tx(true));
+              ++issued;
               ++pr.j;
               *cur = prod_settle(pr, pre, p.B, H, cr);
             }
@@ -595,8 +706,12 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
           // `other`, which this wait acquires, so the copy cannot overtake them
           const uint32_t kp = k - 1;
           const int sp = static_cast<int>(kp % kS);
-          wait_bar(&ps.other[sp], (kp / kS) & 1u, p.err);
-          if (lane == 0) issue_block<BITS, GRP>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen);
+          if (!wait_bar(&ps.other[sp], (kp / kS) & 1u, p.err, abort, p.wait_ns)) {
+            alive = false;
+            break;
+          }
+          if (lane == 0) issue_block<BITS, GRP>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen, extra_tx(true));
+          ++issued;
           ++prod.j;
           prod = prod_settle(prod, pre, p.B, H, cr);
         }
@@ -613,50 +728,66 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
         for (int i = 0; i < 8; ++i) u[hh][i] = 0ull;
       }
       const int g = cs >> 1;                            // V group of channels 16cs..16cs+15
-      const u64 ncorr = pack2(-Tr<BITS, GRP>::kCorrEven, -Tr<BITS, GRP>::kCorrOdd);
       for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
-        wait_bar(kSplit ? &ps.other[stage] : &ps.full[stage], (k / kS) & 1u, p.err);
-        wait_bar(&ps.pfull[pb], (k >> 1) & 1u, p.err);
+        if (!wait_bar(kSplit ? &ps.other[stage] : &ps.full[stage], (k / kS) & 1u, p.err, abort, p.wait_ns)) {
+          alive = false;
+          break;
+        }
+        ++landed;
+        if (!wait_bar(&ps.pfull[pb], (k >> 1) & 1u, p.err, abort, p.wait_ns)) {
+          alive = false;
+          break;
+        }
         const Stage& st = ps.st[stage];
         const int nvalid = min(kTB, len - j * kTB);
 
         // scores of token `lane`: sum the eight channel-slice partials
-        float s[kG] = {0.f, 0.f, 0.f, 0.f};
+        u64 s01 = 0ull, s23 = 0ull;                     // heads (0, 1) and (2, 3)
         const float* part = ps.part[pb];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float4 v = *reinterpret_cast<const float4*>(part + part_index(lane, i));
-          s[0] += v.x;
-          s[1] += v.y;
-          s[2] += v.z;
-          s[3] += v.w;
+          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(part + part_index(lane, i));
+          s01 = add2(s01, v.x);
+          s23 = add2(s23, v.y);
         }
+        float s[kG] = {lo_f(s01), hi_f(s01), lo_f(s23), hi_f(s23)};
         __syncwarp();
         if (lane == 0) mbar_arrive(&ps.pempty[pb]);
 
-        // online softmax over the block (log2 units)
+        // online softmax over the block (log2 units).  The reference m of a
+        // head moves only when a block's maximum exceeds it by more than
+        // kLazy (always on the first block, where m = -inf); otherwise the
+        // block's exponentials are taken against the old reference and stay
+        // below 2^kLazy.  Any reference gives the same u / z in exact
+        // arithmetic (the block rule with a stale but consistent m), and the
+        // partials carry the reference the merge rescales by.
         const bool valid = lane < nvalid;
-        float a[kG], pr[kG];
+        float pr[kG], bm[kG];
         bool grow = false;
 #pragma unroll
         for (int hh = 0; hh < kG; ++hh) {
           s[hh] = valid ? s[hh] : -INFINITY;
-          const float mn = fmaxf(m[hh], warp_max(s[hh]));
-          grow |= mn > m[hh];
-          a[hh] = ex2(m[hh] - mn);                      // 0 on the first block (m = -inf)
-          pr[hh] = valid ? ex2(s[hh] - mn) : 0.f;
-          z[hh] = fmaf(a[hh], z[hh], pr[hh]);
-          m[hh] = mn;
+          bm[hh] = warp_max(s[hh]);
+          grow |= bm[hh] > m[hh] + kLazy;
         }
         if (grow) {                                     // warp-uniform
 #pragma unroll
           for (int hh = 0; hh < kG; ++hh) {
-            const u64 a2 = pack2(a[hh], a[hh]);
+            const float mn = fmaxf(m[hh], bm[hh]);
+            const float a = ex2(m[hh] - mn);            // 0 on the first block (m = -inf)
+            z[hh] *= a;
+            m[hh] = mn;
+            const u64 a2 = pack2(a, a);
 #pragma unroll
             for (int i = 0; i < 8; ++i) u[hh][i] = mul2(u[hh][i], a2);
           }
+        }
+#pragma unroll
+        for (int hh = 0; hh < kG; ++hh) {
+          pr[hh] = valid ? ex2(s[hh] - m[hh]) : 0.f;
+          z[hh] += pr[hh];
         }
         if (GRP == 32) {
           // p' = p * s_v of this lane's token for each V group, as (p', p') pairs
@@ -681,14 +812,11 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
         for (int it = 0; it < kTB / 4; ++it) {
           const int t = block_token<GRP>(it, ts);
           const float4 p4 = *reinterpret_cast<const float4*>(&ps.pv[t][GRP == 32 ? 4 * g : 0]);
+          // (code - qmax) eps exactly, so a zero code contributes exactly zero
           u64 f[8];
-          code_pairs<BITS>(st.vc, t, cs, f);
+          v_offsets<BITS>(st.vc, t, cs, f);
           const u64 pp[kG] = {pack2(p4.x, p4.x), pack2(p4.y, p4.y), pack2(p4.z, p4.z),
                               pack2(p4.w, p4.w)};
-          // f - (1 + qmax eps) = (code - qmax) eps exactly, so a zero code
-          // contributes exactly zero
-#pragma unroll
-          for (int i = 0; i < 8; ++i) f[i] = add2(f[i], ncorr);
           if (GRP == 8) {
             // the scales of V groups 2 cs and 2 cs + 1 (channels 16 cs .. +7,
             // +8 .. +15); zero past the length, where the stage holds stale
@@ -714,7 +842,8 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
             Prod pr = *cur;
             if (pr.valid) {
               fence_proxy_async();
-              issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, false);
+              issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, false, 0u);
+              ++issued;
               ++pr.j;
               *cur = prod_settle(pr, pre, p.B, H, cr);
             }
@@ -724,6 +853,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
         }
       }
 
+      if (!alive) break;
       // the pair's state for the segment: z summed over the token lanes, u
       // over the four token groups; lanes with ts = 0 hold channels 16cs..
 #pragma unroll
@@ -738,8 +868,9 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
         float uf[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          // u carries a factor eps of the channel: scale it back
-          float x = lo_f(u[hh][i]) * Tr<BITS, GRP>::kInvEpsEven, y = hi_f(u[hh][i]) * Tr<BITS, GRP>::kInvEpsOdd;
+          // u carries the factor eps of its slot: scale it back
+          float x = lo_f(u[hh][i]) * VSlot<BITS>::inv_eps(2 * i);
+          float y = hi_f(u[hh][i]) * VSlot<BITS>::inv_eps(2 * i + 1);
           x += __shfl_xor_sync(0xffffffffu, x, 8);
           y += __shfl_xor_sync(0xffffffffu, y, 8);
           x += __shfl_xor_sync(0xffffffffu, x, 16);
@@ -769,6 +900,14 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
     }
     first = false;
     seg = next_seg(seg, pre, p.B, H, cr);
+  }
+  if (!alive && lane == 0) {
+    // a wait ran out: nothing of this pair's segment is written; copies this
+    // warp issued whose completion it has not seen are waited for (bounded)
+    // so none still writes shared memory when the CTA exits
+    const bool issuer = kSplit || is_s;
+    for (uint32_t kk = landed; issuer && kk < issued; ++kk)
+      drain_bar(kSplit && !is_s ? &ps.other[kk % kS] : &ps.full[kk % kS], (kk / kS) & 1u);
   }
 }
 
@@ -852,6 +991,9 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   p.force_partial = a.win_lengths != nullptr;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
+  p.wait_ns = a.test_wait_ns ? a.test_wait_ns : 2000000000ull;
+  p.lose_worker = a.test_lose_block >= 0 ? 0 : -1;
+  p.lose_block = a.test_lose_block;
   const cudaError_t le = launch_pdl(kernel, dim3(ctas), dim3(threads), smem, s, p);
   if (le != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();

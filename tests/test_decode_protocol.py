@@ -4,11 +4,15 @@ One warp pair of `decode_kernel`: the S-warp (scores) and the V-warp
 (values) consume a pair-private ring of stages, each holding one 32-token
 block's K half (K codes and scales, read by the S-warp alone) and V half
 (read by the V-warp alone), and hand each block's partial scores from S to V
-through two alternating buffers (`pfull` / `pempty`).  Two refill protocols
-exist, chosen per variant:
+through one or two alternating buffers (`pfull` / `pempty`).  Three refill
+protocols are modelled:
 
 * whole -- the S-warp refills the whole stage of block k - 1 after its block
   k, once the V-warp has released that stage (`other`);
+* whole_v -- the V-warp, the last reader of every stage, refills the whole
+  stage of block k right after its own last read of it (no release
+  barrier: the S-warp's last read of the stage came before its `pfull`
+  arrive, which the V-warp waited for);
 * split -- each warp refills its own half of a stage right after its own
   last read of it, on its own barrier (`full` for K, `other` for V).
 
@@ -41,14 +45,15 @@ class Bar:
 
 
 class Pair:
-    def __init__(self, n_blocks, n_stages, split, seed, lag, drop=None, shift=None):
-        self.n, self.ks, self.split = n_blocks, n_stages, split
+    def __init__(self, n_blocks, n_stages, protocol, seed, lag, drop=None, shift=None, n_pbufs=2):
+        self.n, self.ks, self.protocol, self.nb = n_blocks, n_stages, protocol, n_pbufs
+        self.split = protocol == "split"
         self.rng, self.lag, self.drop, self.shift = random.Random(seed), lag, drop, shift
         self.bars = {}
         for s in range(n_stages):
             self.bars[("full", s)] = Bar(1)
             self.bars[("other", s)] = Bar(1)
-        for i in range(2):
+        for i in range(n_pbufs):
             self.bars[("pfull", i)] = Bar(1)
             self.bars[("pempty", i)] = Bar(1)
         self.ver = {}                      # buffer -> block it holds
@@ -89,24 +94,24 @@ class Pair:
         return [("wait", bar, k + (self.shift == name))]
 
     def s_warp(self):
-        n, ks = self.n, self.ks
+        n, ks, nb = self.n, self.ks, self.nb
         for s in range(min(ks, n)):
             if self.split:
                 yield ("do", lambda s=s: self.issue(("K", s), s, {"S"}, ("full", s)))
-            else:
+            elif self.protocol == "whole":
                 yield ("do", lambda s=s: self.issue_whole(s, s))
         for k in range(n):
             st = k % ks
             yield from self.wait("s_full", ("full", st), k // ks)
             yield ("do", lambda k=k, st=st: self.use(("K", st), k, "S"))
-            if k >= 2:
-                yield from self.wait("pempty", ("pempty", k & 1), (k - 2) // 2)
-            yield ("do", lambda k=k: self.write(("P", k & 1), k, {"V"}, "S"))
-            yield ("arrive", ("pfull", k & 1))
+            if k >= nb:
+                yield from self.wait("pempty", ("pempty", k % nb), (k - nb) // nb)
+            yield ("do", lambda k=k: self.write(("P", k % nb), k, {"V"}, "S"))
+            yield ("arrive", ("pfull", k % nb))
             if self.split:
                 if k + ks < n:
                     yield ("do", lambda k=k, st=st: self.issue(("K", st), k + ks, {"S"}, ("full", st)))
-            elif k > 0 and k - 1 + ks < n:
+            elif self.protocol == "whole" and k > 0 and k - 1 + ks < n:
                 sp = (k - 1) % ks
                 yield from self.wait("release", ("other", sp), (k - 1) // ks)
                 yield ("do", lambda k=k, sp=sp: self.issue_whole(sp, k - 1 + ks))
@@ -121,21 +126,30 @@ class Pair:
         self.copies.append((buf, block, ("full", stage)))
         self.bars[("full", stage)].tx += 1
 
+    def v_wait_full(self, k, st):
+        # the V-warp's wait on the stage barrier (its own half's in split)
+        return self.wait("v_full", ("other", st) if self.split else ("full", st), k // self.ks)
+
     def v_warp(self):
-        n, ks = self.n, self.ks
-        if self.split:
-            for s in range(min(ks, n)):
+        n, ks, nb = self.n, self.ks, self.nb
+        for s in range(min(ks, n)):
+            if self.split:
                 yield ("do", lambda s=s: self.issue(("V", s), s, {"V"}, ("other", s)))
+            elif self.protocol == "whole_v":
+                yield ("do", lambda s=s: self.issue_whole(s, s))
         for k in range(n):
             st = k % ks
-            yield from self.wait("v_full", ("other", st) if self.split else ("full", st), k // ks)
-            yield from self.wait("pfull", ("pfull", k & 1), k // 2)
-            yield ("do", lambda k=k: self.use(("P", k & 1), k, "V"))
-            yield ("arrive", ("pempty", k & 1))
+            yield from self.v_wait_full(k, st)
+            yield from self.wait("pfull", ("pfull", k % nb), k // nb)
+            yield ("do", lambda k=k: self.use(("P", k % nb), k, "V"))
+            yield ("arrive", ("pempty", k % nb))
             yield ("do", lambda k=k, st=st: self.use(("V", st), k, "V"))
             if self.split:
                 if k + ks < n:
                     yield ("do", lambda k=k, st=st: self.issue(("V", st), k + ks, {"V"}, ("other", st)))
+            elif self.protocol == "whole_v":
+                if k + ks < n:
+                    yield ("do", lambda k=k, st=st: self.issue_whole(st, k + ks))
             else:
                 yield ("arrive", ("other", st))
 
@@ -180,13 +194,15 @@ class Pair:
 
 
 CASES = [(1, 3), (2, 3), (3, 3), (4, 3), (7, 3), (28, 3), (1, 2), (5, 2), (28, 2)]
+PROTOCOLS = ["whole", "whole_v", "split"]
 
 
-@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
+@pytest.mark.parametrize("n_pbufs", [1, 2])
+@pytest.mark.parametrize("protocol", PROTOCOLS)
 @pytest.mark.parametrize("n_blocks,n_stages", CASES)
-def test_protocol_holds(split, n_blocks, n_stages):
+def test_protocol_holds(protocol, n_blocks, n_stages, n_pbufs):
     for seed in range(12):
-        Pair(n_blocks, n_stages, split, seed, lag=(seed % 4) * 0.3).run()
+        Pair(n_blocks, n_stages, protocol, seed, lag=(seed % 4) * 0.3, n_pbufs=n_pbufs).run()
 
 
 # In the whole protocol the V-warp's wait on the stage barrier is implied by
@@ -194,28 +210,31 @@ def test_protocol_holds(split, n_blocks, n_stages):
 # on that same barrier completed, and acquire/release order is transitive.
 # The kernel keeps the direct wait (it returns at once); the model shows it is
 # not load-bearing, so only the split protocol lists it as needed.
-WAITS = {False: ["s_full", "pfull", "pempty", "release"], True: ["s_full", "v_full", "pfull", "pempty"]}
+WAITS = {"whole": ["s_full", "pfull", "pempty", "release"], "whole_v": ["s_full", "pfull", "pempty"],
+         "split": ["s_full", "v_full", "pfull", "pempty"]}
 
 
-@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
-def test_every_wait_is_needed(split):
-    for name in WAITS[split]:
+@pytest.mark.parametrize("n_pbufs", [1, 2])
+@pytest.mark.parametrize("protocol", PROTOCOLS)
+def test_every_wait_is_needed(protocol, n_pbufs):
+    for name in WAITS[protocol]:
         failed = False
         for n_blocks, n_stages in [(7, 3), (6, 2), (28, 3)]:
             for seed in range(60):
                 try:
-                    Pair(n_blocks, n_stages, split, seed, lag=(seed % 4) * 0.3, drop=name).run()
+                    Pair(n_blocks, n_stages, protocol, seed, lag=(seed % 4) * 0.3, drop=name, n_pbufs=n_pbufs).run()
                 except AssertionError:
                     failed = True
                     break
             if failed:
                 break
-        assert failed, f"leaving out the {name} wait went unnoticed ({'split' if split else 'whole'})"
+        assert failed, f"leaving out the {name} wait went unnoticed ({protocol}, {n_pbufs} partial buffers)"
 
 
-@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
-def test_every_phase_is_right(split):
-    for name in WAITS[split]:
+@pytest.mark.parametrize("n_pbufs", [1, 2])
+@pytest.mark.parametrize("protocol", PROTOCOLS)
+def test_every_phase_is_right(protocol, n_pbufs):
+    for name in WAITS[protocol]:
         with pytest.raises(AssertionError):
             for seed in range(10):
-                Pair(7, 3, split, seed, lag=0.3, shift=name).run()
+                Pair(7, 3, protocol, seed, lag=0.3, shift=name, n_pbufs=n_pbufs).run()

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle as O
-from tests.gpu_util import DEV, assert_head_packed_equal, check_rows, to_dev
+from tests.gpu_util import DEV, assert_head_packed_equal, check_rows, check_rows_rounded, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -79,7 +79,14 @@ def _run_steps(sm, b_, hq, hkv, n_cap, d, start, steps, bits, group, in_dtype=to
                 assert_head_packed_equal(cache, b, h, pk, pv)
                 kh, vh = O.unpack_matrix(pk), O.unpack_matrix(pv)
                 want = O.attend_gqa_heads(qv[b, h * grp:(h + 1) * grp, 0], kh, vh, n, 1.0)
-                check_rows(o[b, h * grp:(h + 1) * grp, 0], want, vh, f"step {s} b{b} h{h} len {n}")
+                got, what = o[b, h * grp:(h + 1) * grp, 0], f"step {s} b{b} h{h} len {n}"
+                if q_dtype == torch.bfloat16:
+                    # a short sequence's row can sit near max|V| (one key: the
+                    # row is that key's value), where the bf16 output's own
+                    # rounding exceeds the tolerance: check the rounding interval
+                    check_rows_rounded(got, want, 2e-3 * float(np.abs(vh[:n]).max()), what)
+                else:
+                    check_rows(got, want, vh[:n], what)
         lens = lens + 1
     return crossed
 

@@ -176,7 +176,10 @@ def _check_gqa(sm, q, k, v, lens, bits, group, scale, q_dtype=torch.bfloat16, sp
         want, pk, pv, vh = oracle_rows(rows, k[b, h], v[b, h], bits, group, int(lens[b]), scale)
         assert_head_packed_equal(cache, b, h, pk, pv)
         got = o[b, h * grp:(h + 1) * grp].reshape(grp * lq, d)
-        check_rows(got, want, vh, f"b{b} h{h}")
+        if q_dtype == torch.bfloat16:
+            check_rows_rounded(got, want, 2e-3 * float(np.abs(vh).max()), f"b{b} h{h}")
+        else:
+            check_rows(got, want, vh, f"b{b} h{h}")
     return o
 
 

@@ -19,6 +19,8 @@ import numpy as np
 import pytest
 import torch
 
+from tests.gpu_util import bf16_rounding_gap
+
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda:0"
@@ -56,7 +58,7 @@ def _noalloc(sm, cache, qd, ld, out, splits=0):
 
 def _oracle_check(cache_k, cache_v, qd, lens, got, heads):
     """The noalloc output of the sampled heads against the float64 oracle,
-    within 2e-3 * max|V_hat| of the head."""
+    within 2e-3 * max|V_hat| of the head (beyond the bf16 output's rounding)."""
     import oracle as O
     q = qd.float().cpu().numpy()
     o = got.float().cpu().numpy()
@@ -67,9 +69,12 @@ def _oracle_check(cache_k, cache_v, qd, lens, got, heads):
         pk, pv = O.pack_k(cache_k[b, h], 4, 32), O.pack_v(cache_v[b, h], 4, 32)
         kh, vh = O.unpack_matrix(pk), O.unpack_matrix(pv)
         want = O.attend_gqa_heads(q[b, h * grp:(h + 1) * grp, 0], kh, vh, n, 1.0)
-        err = float(np.abs(o[b, h * grp:(h + 1) * grp, 0] - want).max())
+        # the bf16 output through its rounding interval: a one-token
+        # sequence's row is that token's value, near max|V|, where the
+        # output's own rounding exceeds the tolerance
+        gap = float(bf16_rounding_gap(o[b, h * grp:(h + 1) * grp, 0], want).max())
         tol = 2e-3 * float(np.abs(vh[:n]).max())
-        assert err <= tol, (b, h, err, tol)
+        assert gap <= tol, (b, h, gap, tol)
 
 
 def test_noalloc_two_calls_match_attend(sm):
