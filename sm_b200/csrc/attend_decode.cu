@@ -115,7 +115,8 @@ struct PairSmem {
   unsigned long long pfull[2];        // S-warp wrote part[i]
   unsigned long long pempty[2];       // V-warp read part[i]
   int abort;                          // a wait of this pair ran out: both warps stop
-  int pad_[3];
+  unsigned int issued[2];             // copies each warp issued (lane 0 counts): drained on an abort
+  int pad_;
 };
 
 static_assert(sizeof(Stage<4, 32>) % 16 == 0 && sizeof(Stage<8, 32>) % 16 == 0 &&
@@ -217,33 +218,28 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// Bounded wait of one warp on a phase of `bar`.  Returns true once the phase
-// completed.  Returns false when the pair's abort flag is up (the other warp
-// gave up), or after limit_ns: then it raises the flag itself and records
-// KVQ_ERR_TIMEOUT.  So one lost completion ends the pair's work within one
-// limit, and every later wait of the pair returns at once.
+// Bounded wait on a phase of `bar`: true once the phase completed.  It gives
+// up -- returns false -- when the pair's abort flag is up (the other warp gave
+// up), or after limit_ns, when it raises the flag itself and records
+// KVQ_ERR_TIMEOUT.  Callers go on either way (their next shared-memory reads
+// may then see stale data, which is harmless); each warp checks the flag once
+// per block and leaves its loop, so one lost completion ends the pair's work
+// within one limit and every later wait returns at once.
 __device__ __forceinline__ bool wait_bar(unsigned long long* bar, uint32_t parity, unsigned int* err,
                                          volatile int* abort, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  bool ok = false;
-  if (!*abort) {
-    const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-      if (mbar_try_wait_sleep(bar, parity)) {
-        ok = true;
-        break;
-      }
-      if ((it & 7u) == 0) {
-        if (*abort) break;
-        if (globaltimer() - t0 > limit_ns) {
-          *abort = 1;
-          record_error(err, KVQ_ERR_TIMEOUT);
-          break;
-        }
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 7u) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        *abort = 1;
+        record_error(err, KVQ_ERR_TIMEOUT);
+        return false;
       }
     }
   }
-  return __all_sync(0xffffffffu, ok);
 }
 
 // After an abort: wait (at most about two seconds) for a bulk copy this warp
@@ -536,6 +532,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       mbar_init(&ps.pempty[i], 1);
     }
     ps.abort = 0;
+    ps.issued[0] = ps.issued[1] = 0;
   }
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
@@ -578,12 +575,12 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
     }
   };
   // Copies this warp issued (whole refill: the S-warp's blocks; split: each
-  // warp's halves, counted by lane 0) and the waits on them that completed:
-  // after an abort the difference is drained before the CTA exits.
-  uint32_t issued = 0, landed = 0;
+  // warp's halves), counted in shared memory by lane 0, the issuer: after an
+  // abort the last kS of them are drained before the CTA exits.
+  unsigned int* issued = &ps.issued[is_s ? 0 : 1];
   // the self-test's lost completion: 16 bytes armed that no copy brings
   auto extra_tx = [&](bool k_half) -> uint32_t {
-    return (k_half && worker == p.lose_worker && issued == static_cast<uint32_t>(p.lose_block)) ? 16u : 0u;
+    return (k_half && worker == p.lose_worker && *issued == static_cast<uint32_t>(p.lose_block)) ? 16u : 0u;
   };
   volatile int* abort = &ps.abort;
   if (is_s) load_q(seg);
@@ -592,7 +589,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       Prod pr = prod;
       for (int s = 0; s < kS && pr.valid; ++s) {
         issue_half<BITS, GRP>(p, ps, s, pr.seg.b, pr.seg.h, pr.j, slen, is_s, extra_tx(is_s));
-        ++issued;
+        ++*issued;
         ++pr.j;
         pr = prod_settle(pr, pre, p.B, H, cr);
       }
@@ -600,8 +597,10 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
     }
   } else if (is_s) {
     for (int s = 0; s < kS && prod.valid; ++s) {
-      if (lane == 0) issue_block<BITS, GRP>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen, extra_tx(true));
-      ++issued;
+      if (lane == 0) {
+        issue_block<BITS, GRP>(p, ps, s, prod.seg.b, prod.seg.h, prod.j, slen, extra_tx(true));
+        ++*issued;
+      }
       ++prod.j;
       prod = prod_settle(prod, pre, p.B, H, cr);
     }
@@ -629,11 +628,11 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
-        if (!wait_bar(&ps.full[stage], (k / kS) & 1u, p.err, abort, p.wait_ns)) {
+        if (*abort) {                                    // a wait of this pair ran out
           alive = false;
           break;
         }
-        ++landed;
+        wait_bar(&ps.full[stage], (k / kS) & 1u, p.err, abort, p.wait_ns);
         const Stage& st = ps.st[stage];
 
         // q'' = q * scale * log2e / eps * s_k, as channel pairs (16cs + 2i, +1)
@@ -663,10 +662,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
           }
         }
         // the V-warp must have read this partial buffer's previous block
-        if (k >= 2 && !wait_bar(&ps.pempty[pb], ((k - 2) >> 1) & 1u, p.err, abort, p.wait_ns)) {
-          alive = false;
-          break;
-        }
+        if (k >= 2) wait_bar(&ps.pempty[pb], ((k - 2) >> 1) & 1u, p.err, abort, p.wait_ns);
         float* part = ps.part[pb];
 #pragma unroll 2
         for (int it = 0; it < kTB / 4; ++it) {
@@ -692,10 +688,10 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
           // it with the block kS ahead
           if (lane == 0) {
             Prod pr = *cur;
-            if (pr.valid) {
+            if (pr.valid && !*abort) {                   // no new copy once the pair gave up
               fence_proxy_async();
               issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, true, extra_tx(true));
-              ++issued;
+              ++*issued;
               ++pr.j;
               *cur = prod_settle(pr, pre, p.B, H, cr);
             }
@@ -706,14 +702,15 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
           // `other`, which this wait acquires, so the copy cannot overtake them
           const uint32_t kp = k - 1;
           const int sp = static_cast<int>(kp % kS);
-          if (!wait_bar(&ps.other[sp], (kp / kS) & 1u, p.err, abort, p.wait_ns)) {
-            alive = false;
-            break;
+          // no new copy once the pair gave up: it drains what it issued
+          if (wait_bar(&ps.other[sp], (kp / kS) & 1u, p.err, abort, p.wait_ns)) {
+            if (lane == 0) {
+              issue_block<BITS, GRP>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen, extra_tx(true));
+              ++*issued;
+            }
+            ++prod.j;
+            prod = prod_settle(prod, pre, p.B, H, cr);
           }
-          if (lane == 0) issue_block<BITS, GRP>(p, ps, sp, prod.seg.b, prod.seg.h, prod.j, slen, extra_tx(true));
-          ++issued;
-          ++prod.j;
-          prod = prod_settle(prod, pre, p.B, H, cr);
         }
       }
     } else {
@@ -731,15 +728,12 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       for (int j = seg.jb; j < seg.je; ++j, ++k) {
         const int stage = static_cast<int>(k % kS);
         const int pb = static_cast<int>(k & 1u);
-        if (!wait_bar(kSplit ? &ps.other[stage] : &ps.full[stage], (k / kS) & 1u, p.err, abort, p.wait_ns)) {
+        if (*abort) {                                    // a wait of this pair ran out
           alive = false;
           break;
         }
-        ++landed;
-        if (!wait_bar(&ps.pfull[pb], (k >> 1) & 1u, p.err, abort, p.wait_ns)) {
-          alive = false;
-          break;
-        }
+        wait_bar(kSplit ? &ps.other[stage] : &ps.full[stage], (k / kS) & 1u, p.err, abort, p.wait_ns);
+        wait_bar(&ps.pfull[pb], (k >> 1) & 1u, p.err, abort, p.wait_ns);
         const Stage& st = ps.st[stage];
         const int nvalid = min(kTB, len - j * kTB);
 
@@ -840,10 +834,10 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
           // this warp has read the stage's V half for the last time: refill it
           if (lane == 0) {
             Prod pr = *cur;
-            if (pr.valid) {
+            if (pr.valid && !*abort) {                   // no new copy once the pair gave up
               fence_proxy_async();
               issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, false, 0u);
-              ++issued;
+              ++*issued;
               ++pr.j;
               *cur = prod_settle(pr, pre, p.B, H, cr);
             }
@@ -905,8 +899,11 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
     // a wait ran out: nothing of this pair's segment is written; copies this
     // warp issued whose completion it has not seen are waited for (bounded)
     // so none still writes shared memory when the CTA exits
+    // at most kS copies of a warp are in flight, the last kS it issued (a
+    // phase that already completed passes at once)
     const bool issuer = kSplit || is_s;
-    for (uint32_t kk = landed; issuer && kk < issued; ++kk)
+    const uint32_t n = *issued;
+    for (uint32_t kk = n > kS ? n - kS : 0; issuer && kk < n; ++kk)
       drain_bar(kSplit && !is_s ? &ps.other[kk % kS] : &ps.full[kk % kS], (kk / kS) & 1u);
   }
 }
