@@ -179,9 +179,12 @@ KVQ_API kvq_status kvq_attend_causal(const void* Q, kvq_dtype q_dtype, const kvq
  * Sequence b's new token sits at t = lengths[b] - 1 (lengths count it).  The
  * call re-packs K group t / g of every (b, h) from the caller's float rows of
  * that group -- K scales run along tokens, so a group's scale changes as its
- * tokens arrive -- and packs V row t, in one kernel, then runs kvq_attend with
- * one query row per sequence.  Afterwards the cache holds, for tokens
- * [0, lengths[b]), exactly the bytes kvq_pack of those tokens writes.
+ * tokens arrive -- and packs V row t, then attends with one query row per
+ * sequence as kvq_attend does.  Where the tuned decode kernel runs the attend
+ * (D = 128, four query heads per KV head, 4- or 8-bit, g = 32 or 8) it does
+ * the append itself; other shapes take one append kernel before the attend.
+ * Afterwards the cache holds, for tokens [0, lengths[b]), exactly the bytes
+ * kvq_pack of those tokens writes.
  *   Q, cache, H_q, scale, O, workspace, ws_bytes, splits: as kvq_attend with
  *            Lq = 1 (Q and O [B, H_q, 1, D]; workspace kvq_workspace_size(cache,
  *            H_q, 1, splits) bytes).

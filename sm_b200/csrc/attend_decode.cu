@@ -46,6 +46,7 @@
 #include "f32x2.cuh"
 #include "kvq_internal.cuh"
 #include "plan.cuh"
+#include "quant.cuh"
 
 namespace kvq {
 namespace {
@@ -146,6 +147,13 @@ struct DecodeParams {
   int lose_worker, lose_block;        // self-test of the timeout path: this worker's K copy of its
                                       // lose_block-th block arms 16 bytes more than it brings, so
                                       // that block's barrier never completes; -1: none
+  // decode step (kvq_decode_step): each sequence's new token t = lengths[b] - 1
+  // is appended first -- its K group re-packed from k_tail [B, H, GRP, kD], V
+  // row t from v_new [B, H, kD] -- by the worker that owns the (b, h)'s last
+  // block; nullptr: no append
+  const void* k_tail;
+  const void* v_new;
+  int in_dtype;
 };
 
 // shared memory after the pairs: pre [B + 1], len [B]
@@ -498,10 +506,65 @@ __device__ __forceinline__ void issue_half(const DecodeParams& p, PairSmem<BITS,
   }
 }
 
+// The decode step's append for one (b, h), by the 64 threads of a pair (pt =
+// 0..63 handles channels 2 pt, 2 pt + 1): re-pack K group t / GRP of the new
+// token t from the caller's float rows of that group (rows past t % GRP read
+// as zero, as a whole-cache pack pads a short last group) and pack V row t,
+// into the cache, with the arithmetic of the pack kernels, so the bytes are
+// those a whole-cache pack of tokens [0, t] writes.
+template <int BITS, int GRP>
+__device__ __forceinline__ void append_tail(const DecodeParams& p, int b, int h, int t, int pt) {
+  constexpr int qmax = BITS == 4 ? 7 : 127;
+  const long long head = static_cast<long long>(b) * p.H + h;
+  const int j = t / GRP, nin = t % GRP + 1;
+  const int c = 2 * pt;
+  float x0[GRP], x1[GRP];
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int r = 0; r < GRP; ++r) {
+    x0[r] = 0.f;
+    x1[r] = 0.f;
+    if (r < nin) {
+      const long long e = (head * GRP + r) * kD + c;
+      x0[r] = load_as_f32(p.k_tail, e, p.in_dtype);
+      x1[r] = load_as_f32(p.k_tail, e + 1, p.in_dtype);
+    }
+    a0 = fmaxf(a0, fabsf(x0[r]));
+    a1 = fmaxf(a1, fabsf(x1[r]));
+  }
+  const float s0 = group_scale(a0, qmax), s1 = group_scale(a1, qmax);
+  const float r0 = __frcp_rn(s0), r1 = __frcp_rn(s1);
+  *reinterpret_cast<float2*>(const_cast<float*>(p.k_scales) + head * p.k_scales_head + static_cast<long long>(j) * kD +
+                             c) = make_float2(s0, s1);
+  uint8_t* kc = const_cast<uint8_t*>(p.k_codes) + head * p.k_codes_head;
+#pragma unroll
+  for (int r = 0; r < GRP; ++r) {
+    const unsigned q0 = quant_code(x0[r], s0, r0, qmax), q1 = quant_code(x1[r], s1, r1, qmax);
+    const long long row = static_cast<long long>(j) * GRP + r;
+    if (BITS == 4) kc[row * 64 + pt] = static_cast<uint8_t>(q0 | (q1 << 4));
+    else *reinterpret_cast<uint16_t*>(kc + row * 128 + c) = static_cast<uint16_t>(q0 | (q1 << 8));
+  }
+  // V row t: the GRP / 2 threads of a V group (within one warp) share its max
+  const long long ve = head * kD + c;
+  const float v0 = load_as_f32(p.v_new, ve, p.in_dtype), v1 = load_as_f32(p.v_new, ve + 1, p.in_dtype);
+  float am = fmaxf(fabsf(v0), fabsf(v1));
+#pragma unroll
+  for (int o = 1; o < GRP / 2; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const float sv = group_scale(am, qmax), rv = __frcp_rn(sv);
+  if ((c % GRP) == 0)
+    const_cast<float*>(p.v_scales)[head * p.v_scales_head + static_cast<long long>(t) * (kD / GRP) + c / GRP] = sv;
+  uint8_t* vc = const_cast<uint8_t*>(p.v_codes) + head * p.v_codes_head + static_cast<long long>(t) * (kD * BITS / 8);
+  const unsigned w0 = quant_code(v0, sv, rv, qmax), w1 = quant_code(v1, sv, rv, qmax);
+  if (BITS == 4) vc[pt] = static_cast<uint8_t>(w0 | (w1 << 4));
+  else *reinterpret_cast<uint16_t*>(vc + c) = static_cast<uint16_t>(w0 | (w1 << 8));
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-template <int BITS, int GRP>
+// APPEND: the decode step's form, which appends each sequence's new token
+// first (a separate instantiation, so the plain attend carries none of it).
+template <int BITS, int GRP, bool APPEND>
 __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasPerSm) decode_kernel(DecodeParams p) {
   griddep_wait();
   constexpr int kNP = Tr<BITS, GRP>::kNP, kS = Tr<BITS, GRP>::kS, kThreads = Tr<BITS, GRP>::kThreads;
@@ -546,6 +609,18 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
   if (cr.g0 >= cr.g1) return;
 
   Seg seg = first_seg(pre, p.B, H, cr);
+  if (APPEND) {
+    // decode step: append the new token of every (b, h) whose last block
+    // this pair owns (only this pair reads that block), before any copy of
+    // it is issued; the bulk copies read the cache through the async proxy
+    for (Seg sg = seg; sg.valid; sg = next_seg(sg, pre, p.B, H, cr)) {
+      const int raw = p.lengths[sg.b];
+      if (sg.je == sg.nb && raw >= 1 && raw <= p.N_cap)
+        append_tail<BITS, GRP>(p, sg.b, sg.h, raw - 1, (is_s ? 0 : 32) + lane);
+    }
+    asm volatile("fence.proxy.async;" ::: "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + pair), "r"(64) : "memory");
+  }
   constexpr bool kSplit = Tr<BITS, GRP>::kSplit;
   // Whole refill: the S-warp's copy cursor, in registers.  Split refill:
   // each warp's cursor lives in shared memory and only lane 0 touches it, so
@@ -921,12 +996,13 @@ struct DecodeVariant {
   int pairs, per_sm, threads;
   size_t (*smem)(int B);
   void (*kernel)(DecodeParams);
+  void (*kernel_append)(DecodeParams);
 };
 
 template <int BITS, int GRP>
 DecodeVariant variant_of() {
   return {Tr<BITS, GRP>::kNP, Tr<BITS, GRP>::kCtasPerSm, Tr<BITS, GRP>::kThreads, smem_bytes<BITS, GRP>,
-          decode_kernel<BITS, GRP>};
+          decode_kernel<BITS, GRP, false>, decode_kernel<BITS, GRP, true>};
 }
 
 DecodeVariant variant(const AttendArgs& a) {
@@ -963,7 +1039,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   const int ctas = decode_ctas(a);
   const DecodeVariant v = variant(a);
   const size_t smem = v.smem(a.g.B);
-  auto kernel = v.kernel;
+  auto kernel = a.K_tail_step ? v.kernel_append : v.kernel;
   const int threads = v.threads;
   if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kernel), smem)) return KVQ_ERR_CUDA;
   DecodeParams p{};
@@ -989,6 +1065,9 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
   p.wait_ns = a.test_wait_ns ? a.test_wait_ns : 2000000000ull;
+  p.k_tail = a.K_tail_step;
+  p.v_new = a.V_new_step;
+  p.in_dtype = a.step_dtype;
   p.lose_worker = a.test_lose_block >= 0 ? 0 : -1;
   p.lose_block = a.test_lose_block;
   const cudaError_t le = launch_pdl(kernel, dim3(ctas), dim3(threads), smem, s, p);

@@ -268,6 +268,13 @@ kvq_status kvq_decode_step(const void* Q, kvq_dtype q_dtype, const kvq_cache* ca
   ap.k_scales = cache->k_scales;
   ap.v_codes = cache->v_codes;
   ap.v_scales = cache->v_scales;
+  if (impl == decode_attend_impl()) {
+    // the tuned decode kernel appends the new tokens itself: one launch less
+    a.K_tail_step = K_tail;
+    a.V_new_step = V_new;
+    a.step_dtype = in_dtype;
+    return impl->launch(a, static_cast<cudaStream_t>(stream));
+  }
   if (append_smem_bytes(a.g) > 227 * 1024 || a.g.H_kv > 65535) return KVQ_ERR_UNSUPPORTED;
   const kvq_status ast = launch_append(ap, static_cast<cudaStream_t>(stream));
   if (ast != KVQ_OK) return ast;

@@ -215,6 +215,11 @@ struct AttendArgs {
   // wait is bounded by test_wait_ns; -1 / 0: none, the default limit
   int test_lose_block = -1;
   unsigned long long test_wait_ns = 0;
+  // kvq_decode_step: the new tokens' K group rows and V rows, appended by the
+  // tuned decode kernel itself (nullptr: no append)
+  const void* K_tail_step = nullptr;
+  const void* V_new_step = nullptr;
+  int step_dtype = 0;
 };
 
 // Workspace of an implementation whose packed partials fill `slots` slots of
