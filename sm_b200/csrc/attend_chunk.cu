@@ -284,6 +284,9 @@ __device__ __forceinline__ float row_extreme(const uint32_t (&sr)[64]) {
   return r;
 }
 
+// One instantiation per code width, so each carries one decode path only
+// (a smaller body for the instruction cache the 20 warp roles share).
+template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constant__ CUtensorMap qmap, ChunkParams p) {
   griddep_wait();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -298,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = p.H;
-  const int cb = kD * p.bits / 8;                         // code bytes per token
+  constexpr int cb = kD * BITS / 8;                       // code bytes per token
   const int unit_bytes = kBT * cb + 2048;                 // codes + scales of a K or V half-block
   const uint32_t nu = static_cast<uint32_t>(min(kMaxUnits, kRingBytes / unit_bytes));
 
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
         const unsigned char* u = sm + kOffRing + slot * unit_bytes;
         unsigned char* dst = sm + (is_v ? kOffV : kOffK + (kb & 1u) * 2 * kTileHalf);
         const int nv = min(kBT, slen[c.seg.b] - c.j * kBT);
-        if (p.bits == 4) {
+        if constexpr (BITS == 4) {
           if (is_v) decode_unit4<true>(u, dst, wk, lane, nv);
           else decode_unit4<false>(u, dst, wk, lane, nv);
         } else {
@@ -715,7 +718,8 @@ bool make_q_map(const AttendArgs& a, CUtensorMap* map) {
 kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   const int ctas = chunk_ctas(a);
   const size_t smem = smem_bytes(a.g.B);
-  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(chunk_kernel), smem)) return KVQ_ERR_CUDA;
+  auto kernel = a.g.bits == 4 ? chunk_kernel<4> : chunk_kernel<8>;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kernel), smem)) return KVQ_ERR_CUDA;
   CUtensorMap qmap;
   if (!make_q_map(a, &qmap)) return KVQ_ERR_CUDA;
   ChunkParams p{};
@@ -744,7 +748,7 @@ kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   p.causal = a.causal;
   p.err = error_word();
   if (!p.err) return KVQ_ERR_CUDA;
-  if (launch_pdl(chunk_kernel, dim3(ctas), dim3(kThreads), smem, s, qmap, p) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (launch_pdl(kernel, dim3(ctas), dim3(kThreads), smem, s, qmap, p) != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
 
   MergeArgs m{};
