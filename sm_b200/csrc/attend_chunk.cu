@@ -151,7 +151,7 @@ __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned ch
     }
   }
   const u64 mul = pack2(256.f, 16.f), add = pack2(-263.f, -23.f);
-#pragma unroll
+#pragma unroll 1
   for (int it = 0; it < 2; ++it) {
     const int t = 16 * wk + 8 * it + tt;
     uint4 o[4];
@@ -226,7 +226,7 @@ __device__ __forceinline__ void decode_unit8(const unsigned char* u, unsigned ch
     }
   }
   const u64 sub = pack2(-8388735.f, -8388735.f);
-#pragma unroll 2
+#pragma unroll 1
   for (int it = 0; it < 4; ++it) {
     const int t = 16 * wk + 4 * it + tt;
     uint4 o[2];
@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
           const int nv = p.causal ? min(nv_seq, slen[c.seg.b] - p.Lq + qi + 1 - c.j * kBT) : nv_seq;
           // pass 1: the row's extreme over the valid columns, 64 at a time
           float mx = neg ? INFINITY : -INFINITY;
-#pragma unroll
+#pragma unroll 1
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t sr[64];
             KVQ_LD32_AT(sr, 0, s_col + 64u * hh);
