@@ -201,6 +201,33 @@ def test_gqa_multi_query_rows(sm):
     _check_gqa(sm, q, k, v, lens, 4, 32, 1.0)
 
 
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+@pytest.mark.parametrize("lq", [32, 64])
+def test_chunk_reference_moves_inside_block(sm, sign, lq):
+    """Score spikes placed so that a row's running reference must move in
+    the second, third and fourth 32-column quarter of a 128-token block (and
+    in the first block, after its first quarter), each by more than the lazy
+    threshold: the p already written for the block is rescaled, and O and z
+    of the earlier blocks too.  Both signs of the scale (a negative scale
+    turns the row maximum into a minimum of the raw scores)."""
+    rng = np.random.default_rng(77)
+    b_, hq, hkv, n, d = 2, 8, 2, 520, 128
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    q = (u[None, None, None, :] + 0.05 * rng.standard_normal((b_, hq, lq, d))).astype(np.float32)
+    k = rng.standard_normal((b_, hkv, n, d)).astype(np.float32)
+    v = rng.standard_normal((b_, hkv, n, d)).astype(np.float32)
+    # (token, natural-log score): block 0 quarter 2, block 1 quarter 1,
+    # block 2 quarter 2, block 3 quarter 3; each about 11 log2 units above the last
+    for t, c in ((80, 10.0), (168, 18.0), (326, 26.0), (484, 34.0)):
+        k[:, :, t, :] = sign * c * u
+    lens = np.asarray([520, 300], np.int32)
+    cache = pack_gpu(sm, k, v, 4, 32)
+    assert sm.kernel_name(cache, hq, lq).startswith("chunk")
+    for splits in (0, 1, 3):
+        _check_gqa(sm, q, k, v, lens, 4, 32, sign, splits=splits)
+
+
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("lq", [32, 64])
 def test_chunk_tensor_core_ragged(sm, bits, lq):
