@@ -583,27 +583,45 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
               KVQ_ST32(o_col + 32u * cc, orr);
             }
           }
-          // pass 2: p = exp2(s * qscale - m_ref) as bf16, written over the S columns
+          // pass 2: p = exp2(s * qscale - m_ref) as bf16, written over the S columns.
+          // A block with every row's columns valid (all blocks but a sequence's
+          // last, without the causal mask) takes a loop with no masking; the
+          // choice is warp-wide because the TMEM accesses are.
           const u64 qs2 = pack2(p.qscale, p.qscale), nm2 = pack2(-m_ref, -m_ref);
           u64 z2 = 0ull;
+          if (__all_sync(0xffffffffu, nv >= kBT)) {
 #pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t sr[32];
-            KVQ_LD32(sr, s_col + 32u * cc);
-            tmem_wait_ld();
-            uint32_t pk[16];
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t sr[32];
+              KVQ_LD32(sr, s_col + 32u * cc);
+              tmem_wait_ld();
+              uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const u64 x = fma2(pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), qs2, nm2);
-              float p0 = ex2(lo_f(x)), p1 = ex2(hi_f(x));
-              if (nv < kBT) {
-                p0 = 32 * cc + 2 * e < nv ? p0 : 0.f;
-                p1 = 32 * cc + 2 * e + 1 < nv ? p1 : 0.f;
+              for (int e = 0; e < 16; ++e) {
+                const u64 x = fma2(pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), qs2, nm2);
+                const float p0 = ex2(lo_f(x)), p1 = ex2(hi_f(x));
+                z2 = add2(z2, pack2(p0, p1));
+                pk[e] = pack_bf16(p0, p1);
               }
-              z2 = add2(z2, pack2(p0, p1));
-              pk[e] = pack_bf16(p0, p1);
+              KVQ_ST16(s_col + 16u * cc, pk);
             }
-            KVQ_ST16(s_col + 16u * cc, pk);
+          } else {
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t sr[32];
+              KVQ_LD32(sr, s_col + 32u * cc);
+              tmem_wait_ld();
+              uint32_t pk[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const u64 x = fma2(pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), qs2, nm2);
+                const float p0 = 32 * cc + 2 * e < nv ? ex2(lo_f(x)) : 0.f;
+                const float p1 = 32 * cc + 2 * e + 1 < nv ? ex2(hi_f(x)) : 0.f;
+                z2 = add2(z2, pack2(p0, p1));
+                pk[e] = pack_bf16(p0, p1);
+              }
+              KVQ_ST16(s_col + 16u * cc, pk);
+            }
           }
           z += lo_f(z2) + hi_f(z2);
           tmem_wait_st();

@@ -46,16 +46,21 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // Bounded wait: after about two seconds record KVQ_ERR_TIMEOUT, raise the
 // CTA's abort flag and go on; once the flag is up every later wait of the CTA
 // returns at once, so the kernel always reaches its end (and frees its tensor
-// memory) within a few seconds.
+// memory) within a few seconds.  The flag and the clock are looked at once
+// every 16 polls: a poll is a handful of instructions, the checks twice as
+// many, and waiting warps share the schedulers with working ones.
 __device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, unsigned int* err, volatile int* abort_flag) {
   if (mbar_try(bar, parity)) return;
   const uint64_t t0 = globaltimer();
-  while (!mbar_try(bar, parity)) {
-    if (*abort_flag) return;
-    if (globaltimer() - t0 > 2000000000ull) {
-      record_error(err, KVQ_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return;
+      if (globaltimer() - t0 > 2000000000ull) {
+        record_error(err, KVQ_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return;
+      }
     }
   }
 }
