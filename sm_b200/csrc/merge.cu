@@ -8,9 +8,13 @@
 //
 // Two layouts of the per-worker partial states (a worker is a CTA, or a warp
 // pair of the decode kernel).  Row-major ([slot][row][m, z, u...]), for the
-// few-row decode kernels.  Feature-major ([slot][field][row]), for the
-// many-row chunk kernel: one CTA per (b, h), 32-row chunk and 32-feature
-// slice, lane = row so every partial read is a coalesced 128-byte line.
+// decode and generic kernels: one CTA per (b, h) and row, parts spread over
+// its warps.  Feature-major ([slot][field][row]), for the many-row chunk
+// kernel: one CTA per (b, h), 32-row chunk and 32-feature slice, lane = row
+// so every partial read is a coalesced 128-byte line.  Both load a batch of
+// parts (m, z and the thread's u values) before using any of it and fold the
+// batch into a running state, so a (b, h) split a few ways costs one round
+// trip to memory.
 //
 // The parts of (b, h) are the packed-cache workers that covered it (slots
 // c + b * H_kv + h for the plan's workers c_first..c_last) and, with a
@@ -74,28 +78,49 @@ __device__ __forceinline__ long long part_slot(const MergePlan& p, int i, long l
   return i < p.parts ? p.c_first + i + bh : p.win_slot;
 }
 
-// Order-preserving integer keys, so that shared-memory atomicMax finds a
-// float maximum.
-__device__ __forceinline__ unsigned int order_key(float f) {
-  const unsigned int u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float from_order_key(unsigned int k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+// Folds a batch of parts into a running state (M, Z, U[]) with the same
+// rule: the batch's largest m over parts that exist (k < n) and hold a key
+// (z > 0) becomes the reference if it is larger, the state is scaled by
+// exp(M_old - M) and each part adds exp(m_c - M) * (z_c, u_c).  Every load of
+// the batch was issued before this runs, so a batch costs one round trip.
+template <int PB, int F>
+__device__ __forceinline__ void fold_batch(float& M, float& Z, float (&U)[F], const float (&mc)[PB],
+                                           const float (&zc)[PB], const float (&uc)[PB][F], int n) {
+  float mb = M;
+#pragma unroll
+  for (int k = 0; k < PB; ++k)
+    if (k < n && zc[k] > 0.f) mb = fmaxf(mb, mc[k]);
+  if (mb == -INFINITY) return;                       // no key yet
+  const float sa = expf(M - mb);                     // 0 while M = -inf (Z, U are 0)
+  Z *= sa;
+#pragma unroll
+  for (int j = 0; j < F; ++j) U[j] *= sa;
+  M = mb;
+#pragma unroll
+  for (int k = 0; k < PB; ++k) {
+    if (k < n && zc[k] > 0.f) {
+      const float w = expf(mc[k] - M);
+      Z = fmaf(w, zc[k], Z);
+#pragma unroll
+      for (int j = 0; j < F; ++j) U[j] = fmaf(w, uc[k][j], U[j]);
+    }
+  }
 }
 
-// Row-major merge for (b, h)s of few parts: one CTA per (b, h).  Pass 1
-// spreads the (part, row) pairs over the threads, so each row's largest m
-// takes one round of loads; pass 2 gives each thread one (row, feature) and
-// walks the parts eight loads deep, weighting each part's z and u by
-// exp(m_c - m).
-constexpr int kMergeThreads = 512;
-constexpr int kMaxMergeRows = 64;   // rows per pass; more rows repeat the passes
+// Row-major merge: one CTA per (b, h) and row, `blockDim.x / 32` warps; lane
+// l owns features l + 32 j (D <= 256).  Warp w takes parts w * kRowPB ..
+// + kRowPB - 1 of each round of blockDim.x / 32 * kRowPB parts, loading a
+// part's m, z and the lane's u values together; the warps' states are then
+// combined through shared memory, one feature per thread.
+constexpr int kRowPB = 4;         // parts a warp loads per round
+constexpr int kRowF = 8;          // features per lane
+constexpr int kRowMaxWarps = 8;
 
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams mp) {
+__global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergeParams mp) {
   griddep_wait();
   extern __shared__ int s_pre[];                 // [B + 1]
-  __shared__ unsigned int s_mkey[kMaxMergeRows];
+  __shared__ float s_m[kRowMaxWarps], s_z[kRowMaxWarps];
+  __shared__ float s_u[kRowMaxWarps][256];
   const MergeArgs& a = mp.a;
   if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
   __syncthreads();
@@ -103,132 +128,73 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(MergeParams mp) {
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
   const int D = a.D;
-  const long long row_base = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq;
-  const MergePlan pl = merge_plan(a, s_pre, b, h, mp.err, h == 0 && threadIdx.x == 0);
-  if (pl.zero) {
-    for (int idx = threadIdx.x; idx < a.R * D; idx += blockDim.x)
-      store_from_f32(a.O, row_base * D + idx, 0.f, a.o_dtype);
-    return;
-  }
-  if (pl.skip) return;
-  const int W = D + 2;
-  const long long slot = static_cast<long long>(a.R_pad) * W;
-
-  for (int r0 = 0; r0 < a.R; r0 += kMaxMergeRows) {
-    const int nr = min(kMaxMergeRows, a.R - r0);
-    for (int i = threadIdx.x; i < nr; i += blockDim.x) s_mkey[i] = order_key(-INFINITY);
-    __syncthreads();
-    // pass 1: each row's largest m over the parts with z > 0
-    for (int i = threadIdx.x; i < pl.total * nr; i += blockDim.x) {
-      const int c = i / nr, r = r0 + i % nr;
-      const float* pr = a.partials + part_slot(pl, c, bh) * slot + static_cast<long long>(r) * W;
-      if (pr[1] > 0.f) atomicMax(&s_mkey[r - r0], order_key(pr[0]));
-    }
-    __syncthreads();
-    // pass 2: one (row, feature) per thread
-    for (int idx = threadIdx.x; idx < nr * D; idx += blockDim.x) {
-      const int r = r0 + idx / D, d = idx % D;
-      const float m = from_order_key(s_mkey[r - r0]);
-      float z = 0.f, u = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < pl.total; ++c) {
-        const float* pc = a.partials + part_slot(pl, c, bh) * slot + static_cast<long long>(r) * W;
-        const float zc = pc[1], mc = pc[0], uc = pc[2 + d];
-        if (zc > 0.f) {
-          const float w = expf(mc - m);
-          z = fmaf(w, zc, z);
-          u = fmaf(w, uc, u);
-        }
-      }
-      store_from_f32(a.O, (row_base + r) * D + d, z > 0.f ? u / z : 0.f, a.o_dtype);
-    }
-    __syncthreads();
-  }
-}
-
-// Row-major merge for (b, h)s split into many parts (long sequences): one
-// CTA per (b, h), row and 32-feature slice; warp w takes parts w, w + 8, ...,
-// so the parts are read in one or two rounds of loads.  The parts' largest m
-// is found first (pass 1, then over the warps), then each warp sums its
-// parts' z and u weighted by exp(m_c - m) (pass 2) and warp 0 adds the eight
-// sums.  A lane owns one feature; m and z of a part are one broadcast load.
-constexpr int kMW = 8;            // warps = part groups
-
-__global__ void __launch_bounds__(kMW * 32) merge_parts_kernel(MergeParams mp) {
-  griddep_wait();
-  extern __shared__ int s_pre[];                 // [B + 1]
-  __shared__ float s_m[kMW], s_z[kMW], s_u[kMW][32];
-  const MergeArgs& a = mp.a;
-  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
-  __syncthreads();
-  const int H = a.H_kv;
-  const int bh = blockIdx.x;
-  const int b = bh / H, h = bh % H;
-  const int D = a.D;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r = blockIdx.z;
-  const int d = blockIdx.y * 32 + lane;
-  const bool live = d < D;
+  const int r = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const long long row = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r;
-  const MergePlan pl =
-      merge_plan(a, s_pre, b, h, mp.err, h == 0 && blockIdx.y == 0 && r == 0 && threadIdx.x == 0);
+  const MergePlan pl = merge_plan(a, s_pre, b, h, mp.err, h == 0 && r == 0 && threadIdx.x == 0);
   if (pl.zero) {
-    if (warp == 0 && live) store_from_f32(a.O, row * D + d, 0.f, a.o_dtype);
+    for (int d = threadIdx.x; d < D; d += blockDim.x) store_from_f32(a.O, row * D + d, 0.f, a.o_dtype);
     return;
   }
   if (pl.skip) return;
-  const int W = D + 2;
-  const long long slot = static_cast<long long>(a.R_pad) * W;
-  const long long roff = static_cast<long long>(r) * W;
+  const long long slot = static_cast<long long>(a.R_pad) * (D + 2);
+  const long long roff = static_cast<long long>(r) * (D + 2);
 
-  float m = -INFINITY;
-#pragma unroll 4
-  for (int c = warp; c < pl.total; c += kMW) {
-    const float* pc = a.partials + part_slot(pl, c, bh) * slot + roff;
-    const float zc = pc[1], mc = pc[0];
-    if (zc > 0.f) m = fmaxf(m, mc);
-  }
-  if (lane == 0) s_m[warp] = m;
-  __syncthreads();
+  float M = -INFINITY, Z = 0.f, U[kRowF];
 #pragma unroll
-  for (int w = 0; w < kMW; ++w) m = fmaxf(m, s_m[w]);
-
-  float z = 0.f, u = 0.f;
-#pragma unroll 4
-  for (int c = warp; c < pl.total; c += kMW) {
-    const float* pc = a.partials + part_slot(pl, c, bh) * slot + roff;
-    const float zc = pc[1], mc = pc[0];
-    const float uc = live ? pc[2 + d] : 0.f;
-    if (zc > 0.f) {
-      const float w = expf(mc - m);
-      z = fmaf(w, zc, z);
-      u = fmaf(w, uc, u);
-    }
-  }
-  s_u[warp][lane] = u;
-  if (lane == 0) s_z[warp] = z;
-  __syncthreads();
-  if (warp == 0 && live) {
-    float zt = 0.f, ut = 0.f;
+  for (int j = 0; j < kRowF; ++j) U[j] = 0.f;
+  for (int base = warp * kRowPB; base < pl.total; base += nw * kRowPB) {
+    float mc[kRowPB], zc[kRowPB], uc[kRowPB][kRowF];
 #pragma unroll
-    for (int w = 0; w < kMW; ++w) {
-      zt += s_z[w];
-      ut += s_u[w][lane];
+    for (int k = 0; k < kRowPB; ++k) {
+      const int c = min(base + k, pl.total - 1);   // past the last part: reload it, masked below
+      const float* pc = a.partials + part_slot(pl, c, bh) * slot + roff;
+      mc[k] = pc[0];
+      zc[k] = pc[1];
+#pragma unroll
+      for (int j = 0; j < kRowF; ++j) {
+        const int d = lane + 32 * j;
+        uc[k][j] = d < D ? pc[2 + d] : 0.f;
+      }
     }
-    store_from_f32(a.O, row * D + d, zt > 0.f ? ut / zt : 0.f, a.o_dtype);
+    fold_batch<kRowPB, kRowF>(M, Z, U, mc, zc, uc, pl.total - base);
+  }
+  if (lane == 0) {
+    s_m[warp] = M;
+    s_z[warp] = Z;
+  }
+#pragma unroll
+  for (int j = 0; j < kRowF; ++j) {
+    const int d = lane + 32 * j;
+    if (d < D) s_u[warp][d] = U[j];
+  }
+  __syncthreads();
+  float Mt = -INFINITY;
+  for (int w = 0; w < nw; ++w)
+    if (s_z[w] > 0.f) Mt = fmaxf(Mt, s_m[w]);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float z = 0.f, u = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      if (s_z[w] > 0.f) {
+        const float e = expf(s_m[w] - Mt);
+        z = fmaf(e, s_z[w], z);
+        u = fmaf(e, s_u[w][d], u);
+      }
+    }
+    store_from_f32(a.O, row * D + d, z > 0.f ? u / z : 0.f, a.o_dtype);   // z = 0: a row with no key
   }
 }
-
-constexpr int kFmRows = 32;       // rows per CTA of the feature-major merge
-constexpr int kFmCols = 32;       // features per CTA
-constexpr int kFmThreads = 128;   // 4 warps x 8 features
-constexpr int kFmBatch = 4;       // parts whose weights are held at once
 
 // Feature-major merge: one CTA per (b, h), 32-row chunk and 32-feature
-// slice; lane = row, so every read of a part's field is one coalesced
-// 128-byte line; warp w owns 8 features.  The weights exp(m_c - m) of up to
-// four parts sit in registers and each part's 8 values are loaded together.
-__global__ void __launch_bounds__(kFmThreads, 4) merge_fm_kernel(MergeParams mp) {
+// slice; lane = row, so each field read of a part is one coalesced 128-byte
+// line, and warp w owns features 4w .. 4w + 3 of the slice.  A thread loads
+// m, z and its four u values of up to kFmPB parts in one round.
+constexpr int kFmRows = 32;       // rows per CTA
+constexpr int kFmF = 4;           // features per thread
+constexpr int kFmWarps = 8;       // 8 x 4 = 32 features per CTA
+constexpr int kFmPB = 8;          // parts per round
+
+__global__ void __launch_bounds__(kFmWarps * 32, 3) merge_fm_kernel(MergeParams mp) {
   griddep_wait();
   extern __shared__ int s_pre[];                   // [B + 1]
   const MergeArgs& a = mp.a;
@@ -240,59 +206,45 @@ __global__ void __launch_bounds__(kFmThreads, 4) merge_fm_kernel(MergeParams mp)
   const int b = bh / H, h = bh % H;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = blockIdx.y * kFmRows + lane;
-  const int f0 = blockIdx.z * kFmCols + 8 * warp;
+  const int f0 = blockIdx.z * (kFmWarps * kFmF) + kFmF * warp;
   const long long row = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r;
   const MergePlan pl =
       merge_plan(a, s_pre, b, h, mp.err, h == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0);
   const bool live = r < a.R && f0 < D;
+  const int nf = min(kFmF, D - f0);
   if (pl.zero) {
     if (live)
-      for (int j = 0; j < 8 && f0 + j < D; ++j) store_from_f32(a.O, row * D + f0 + j, 0.f, a.o_dtype);
+      for (int j = 0; j < nf; ++j) store_from_f32(a.O, row * D + f0 + j, 0.f, a.o_dtype);
     return;
   }
   if (pl.skip || !live) return;
   const long long slot_floats = static_cast<long long>(D + 2) * a.R_pad;
   const long long rp = a.R_pad;
-  const float* col = a.partials + r;              // part i of this row: col + part_slot(i) * slot_floats
-  float m = -INFINITY;
-#pragma unroll 4
-  for (int c = 0; c < pl.total; ++c) {
-    const float* part = col + part_slot(pl, c, bh) * slot_floats;
-    const float zc = part[rp], mc = part[0];
-    if (zc > 0.f) m = fmaxf(m, mc);
-  }
-  float z = 0.f, u[8];
+  const float* col = a.partials + r;              // part c of this row: col + part_slot(c) * slot_floats
+  float M = -INFINITY, Z = 0.f, U[kFmF];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) u[j] = 0.f;
-  const int nf = min(8, D - f0);
-  for (int cb = 0; cb < pl.total; cb += kFmBatch) {
-    float wgt[kFmBatch], v[kFmBatch][8];
+  for (int j = 0; j < kFmF; ++j) U[j] = 0.f;
+  for (int base = 0; base < pl.total; base += kFmPB) {
+    float mc[kFmPB], zc[kFmPB], uc[kFmPB][kFmF];
 #pragma unroll
-    for (int k = 0; k < kFmBatch; ++k) {
-      const int c = min(cb + k, pl.total - 1);
+    for (int k = 0; k < kFmPB; ++k) {
+      const int c = min(base + k, pl.total - 1);
       const float* part = col + part_slot(pl, c, bh) * slot_floats;
-      const float zc = part[rp], mc = part[0];
-      wgt[k] = (cb + k < pl.total && zc > 0.f) ? expf(mc - m) : 0.f;
-      z += wgt[k] * (zc > 0.f ? zc : 0.f);
+      mc[k] = part[0];
+      zc[k] = part[rp];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[k][j] = j < nf ? part[(2 + f0 + j) * rp] : 0.f;
+      for (int j = 0; j < kFmF; ++j) uc[k][j] = j < nf ? part[(2 + f0 + j) * rp] : 0.f;
     }
-#pragma unroll
-    for (int k = 0; k < kFmBatch; ++k)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) u[j] = fmaf(wgt[k], v[k][j], u[j]);
+    fold_batch<kFmPB, kFmF>(M, Z, U, mc, zc, uc, pl.total - base);
   }
-  const float inv = z > 0.f ? 1.f / z : 0.f;      // z = 0: a causal row with no visible key
-  if (a.o_dtype == KVQ_BF16 && nf == 8) {
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat162 t = __floats2bfloat162_rn(u[2 * j] * inv, u[2 * j + 1] * inv);
-      o[j] = *reinterpret_cast<const uint32_t*>(&t);
-    }
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + row * D + f0) = make_uint4(o[0], o[1], o[2], o[3]);
+  const float inv = Z > 0.f ? 1.f / Z : 0.f;      // Z = 0: a causal row with no visible key
+  if (a.o_dtype == KVQ_BF16 && nf == kFmF) {
+    const __nv_bfloat162 t0 = __floats2bfloat162_rn(U[0] * inv, U[1] * inv);
+    const __nv_bfloat162 t1 = __floats2bfloat162_rn(U[2] * inv, U[3] * inv);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.O) + row * D + f0) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&t0), *reinterpret_cast<const uint32_t*>(&t1));
   } else {
-    for (int j = 0; j < nf; ++j) store_from_f32(a.O, row * D + f0 + j, u[j] * inv, a.o_dtype);
+    for (int j = 0; j < nf; ++j) store_from_f32(a.O, row * D + f0 + j, U[j] * inv, a.o_dtype);
   }
 }
 
@@ -302,27 +254,25 @@ kvq_status launch_merge(const MergeArgs& a, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(a.B + 1) * sizeof(int);
   const long long bh = static_cast<long long>(a.B) * a.H_kv;
   if (bh > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
-  if (smem > 48 * 1024) return KVQ_ERR_UNSUPPORTED;
+  if (smem > 48 * 1024 || a.D > 256 || a.D < 1) return KVQ_ERR_UNSUPPORTED;
   MergeParams mp{a, error_word()};
   if (!mp.err) return KVQ_ERR_CUDA;
   cudaError_t le;
   if (a.feature_major) {
     const int chunks = (a.R + kFmRows - 1) / kFmRows;
-    const int slices = (a.D + kFmCols - 1) / kFmCols;
+    const int slices = (a.D + kFmWarps * kFmF - 1) / (kFmWarps * kFmF);
     if (chunks > 65535 || slices > 65535 || (a.D % 8) != 0) return KVQ_ERR_UNSUPPORTED;
     le = launch_pdl(merge_fm_kernel, dim3(static_cast<unsigned>(bh), static_cast<unsigned>(chunks),
                                           static_cast<unsigned>(slices)),
-                    dim3(kFmThreads), smem, s, mp);
-  } else if (a.ctas >= 8 * bh) {
-    // on average eight or more workers per (b, h): split the parts over warps
-    if (a.R > 65535) return KVQ_ERR_UNSUPPORTED;
-    le = launch_pdl(merge_parts_kernel,
-                    dim3(static_cast<unsigned>(bh), static_cast<unsigned>((a.D + 31) / 32), static_cast<unsigned>(a.R)),
-                    dim3(kMW * 32), smem, s, mp);
+                    dim3(kFmWarps * 32), smem, s, mp);
   } else {
-    const long long work = static_cast<long long>(a.R) * a.D;
-    const int threads = work >= kMergeThreads ? kMergeThreads : static_cast<int>((work + 31) / 32 * 32);
-    le = launch_pdl(merge_kernel, dim3(static_cast<unsigned>(bh)), dim3(threads), smem, s, mp);
+    // warps per row: enough for the workers' average share of a (b, h) (plus
+    // the ragged ends and a window part) in one round
+    if (a.R > 65535) return KVQ_ERR_UNSUPPORTED;
+    const long long parts = (static_cast<long long>(a.ctas) + bh - 1) / bh + 2;
+    const long long nw = std::min<long long>(kRowMaxWarps, std::max<long long>(1, (parts + kRowPB - 1) / kRowPB));
+    le = launch_pdl(merge_rows_kernel, dim3(static_cast<unsigned>(bh), static_cast<unsigned>(a.R)),
+                    dim3(static_cast<unsigned>(nw * 32)), smem, s, mp);
   }
   if (le != cudaSuccess) return KVQ_ERR_CUDA;
   count_launch();
