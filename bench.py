@@ -134,6 +134,7 @@ PROFILE_FOR = {
     ("decode_gqa", 4, 32): "attend_decode_gqa_b32_ctx4096.md",
     ("decode_gqa", 8, 32): "attend_decode_gqa_b32_ctx4096_8bit.md",
     ("chunk", 4, 32): "attend_chunk_b4_lq64_ctx16384.md",
+    ("chunk", 8, 32): "attend_chunk_b4_lq64_ctx16384_8bit.md",
 }
 
 
