@@ -251,6 +251,34 @@ def distribution(us):
             "all": [round(float(x), 3) for x in a]}
 
 
+def copy_rows_h2d(dst, src, stream) -> None:
+    """Pinned host rows into a strided device view with one pitched copy
+    (cudaMemcpy2DAsync: the copy engine alone).  `dst` is the last rows of a
+    contiguous [B, H, W, D] device tensor (dst = t[:, :, -L:]), `src` a
+    contiguous [B, H, L, D] pinned host tensor.  torch's copy_ into such a
+    view stages the rows and runs an elementwise kernel on the copy stream,
+    which cannot start while an attend kernel holds every SM."""
+    import ctypes
+    import torch
+    global _CUDART
+    if "_CUDART" not in globals():
+        import nvidia.cuda_runtime as rt
+        lib = ctypes.CDLL(os.path.join(list(rt.__path__)[0], "lib", "libcudart.so.12"))
+        fn = lib.cudaMemcpy2DAsync
+        fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_size_t,
+                       ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+        fn.restype = ctypes.c_int
+        _CUDART = fn
+    B_, H_, L_, D_ = src.shape
+    assert dst.shape == src.shape and src.is_contiguous() and dst.stride(3) == 1
+    assert dst.stride(0) == H_ * dst.stride(1) and dst.stride(2) == D_
+    es = src.element_size()
+    rc = _CUDART(ctypes.c_void_p(dst.data_ptr()), dst.stride(1) * es, ctypes.c_void_p(src.data_ptr()),
+                 L_ * D_ * es, L_ * D_ * es, B_ * H_, 1, ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"cudaMemcpy2DAsync failed: {rc}")
+
+
 class L2Flush:
     """Writes a buffer twice the size of L2 (at least 256 MB), outside any
     timed region, so the next launch finds none of its inputs in L2."""
@@ -518,7 +546,7 @@ def run_kvq(args, rank, world, local_rank):
                 jn = (i + 1) & 1
                 q_in[jn].copy_(q_host, non_blocking=True)
                 if append:
-                    k_in[jn][:, :, -Lq:].copy_(kv_host_k, non_blocking=True)
+                    copy_rows_h2d(k_in[jn][:, :, -Lq:], kv_host_k, copy_stream)
                     v_in[jn].copy_(kv_host_v, non_blocking=True)
                 ready[jn].record(copy_stream)
 
@@ -529,7 +557,7 @@ def run_kvq(args, rank, world, local_rank):
         with torch.cuda.stream(copy_stream):
             q_in[0].copy_(q_host, non_blocking=True)
             if append:
-                k_in[0][:, :, -Lq:].copy_(kv_host_k, non_blocking=True)
+                copy_rows_h2d(k_in[0][:, :, -Lq:], kv_host_k, copy_stream)
                 v_in[0].copy_(kv_host_v, non_blocking=True)
             ready[0].record(copy_stream)
         for i in range(n):
