@@ -518,17 +518,28 @@ __device__ __forceinline__ void append_tail(const DecodeParams& p, int b, int h,
   const long long head = static_cast<long long>(b) * p.H + h;
   const int j = t / GRP, nin = t % GRP + 1;
   const int c = 2 * pt;
+  // the group's rows of channels c, c + 1; the dtype branch sits outside the
+  // row loop so the 2 GRP loads go out back to back (one round trip)
   float x0[GRP], x1[GRP];
+  const long long e0 = head * GRP * kD + c;
+  if (p.in_dtype == KVQ_F32) {
+    const float* src = static_cast<const float*>(p.k_tail) + e0;
+#pragma unroll
+    for (int r = 0; r < GRP; ++r) {
+      x0[r] = r < nin ? src[r * kD] : 0.f;
+      x1[r] = r < nin ? src[r * kD + 1] : 0.f;
+    }
+  } else {
+    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.k_tail) + e0;
+#pragma unroll
+    for (int r = 0; r < GRP; ++r) {
+      x0[r] = r < nin ? __bfloat162float(src[r * kD]) : 0.f;
+      x1[r] = r < nin ? __bfloat162float(src[r * kD + 1]) : 0.f;
+    }
+  }
   float a0 = 0.f, a1 = 0.f;
 #pragma unroll
   for (int r = 0; r < GRP; ++r) {
-    x0[r] = 0.f;
-    x1[r] = 0.f;
-    if (r < nin) {
-      const long long e = (head * GRP + r) * kD + c;
-      x0[r] = load_as_f32(p.k_tail, e, p.in_dtype);
-      x1[r] = load_as_f32(p.k_tail, e + 1, p.in_dtype);
-    }
     a0 = fmaxf(a0, fabsf(x0[r]));
     a1 = fmaxf(a1, fabsf(x1[r]));
   }
