@@ -104,7 +104,7 @@ struct ChunkParams {
   long long k_codes_head, k_scales_head, v_codes_head, v_scales_head;
   float qscale;                          // scale * log2(e)
   __nv_bfloat16* O;
-  float* partials;                       // [slots][kD + 2][R]: m, z, u (feature-major)
+  float* partials;                       // [slots][R / 32][kD + 2][32]: m, z, u (feature-major)
   int ctas;
   int force_partial;                     // a window follows: no CTA writes output rows
   int causal;                            // query i of Lq reads keys [0, len - Lq + i] only
@@ -636,10 +636,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
             const long long head = static_cast<long long>(c.seg.b) * H + c.seg.h;
             const long long row = (static_cast<long long>(c.seg.b) * H * p.G + static_cast<long long>(c.seg.h) * p.G) *
                                       p.Lq + tile * 128 + r;
-            float* part = p.partials + (static_cast<long long>(blockIdx.x) + head) * (kD + 2) * p.R + tile * 128 + r;
+            // the slot's rows in 32-row chunks, each chunk's fields contiguous
+            // (field f of row rr at (rr / 32) * (kD + 2) * 32 + f * 32 + rr % 32):
+            // this warp's 32 rows are one chunk, written as 130 whole lines
+            const int rr = tile * 128 + r;
+            float* part = p.partials + (static_cast<long long>(blockIdx.x) + head) * (kD + 2) * p.R +
+                          static_cast<long long>(rr >> 5) * (kD + 2) * 32 + (rr & 31);
             if (!whole) {
               part[0] = m_ref * kLn2;
-              part[p.R] = z;
+              part[32] = z;
             }
             // z = 0: a causal row with no visible key (length < Lq, reported by the merge)
             const float inv = z > 0.f ? 1.f / z : 0.f;
@@ -659,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_kernel(const __grid_constan
                   dst[qq] = make_uint4(ob[4 * qq], ob[4 * qq + 1], ob[4 * qq + 2], ob[4 * qq + 3]);
               } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) part[static_cast<long long>(2 + 32 * cc + e) * p.R] = __uint_as_float(orr[e]);
+                for (int e = 0; e < 32; ++e) part[(2 + 32 * cc + e) * 32] = __uint_as_float(orr[e]);
               }
             }
             tc_fence_before();
@@ -787,7 +792,8 @@ kvq_status chunk_launch(const AttendArgs& a, cudaStream_t s) {
   m.causal = a.causal;
   m.feature_major = true;
   const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(ctas, a.g.B, a.g.H_kv)),
-                                   static_cast<long long>(kD + 2) * p.R, 1, p.R, &m, s);
+                                   static_cast<long long>(kD + 2) * p.R, 1, static_cast<long long>(kD + 2) * 32, 32,
+                                   &m, s);
   if (ws != KVQ_OK) return ws;
   return launch_merge(m, s);
 }

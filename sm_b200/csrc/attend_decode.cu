@@ -1101,7 +1101,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   m.G = kG;
   m.Lq = 1;
   const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(m.ctas, a.g.B, a.g.H_kv)),
-                                   kG * (kD + 2), kD + 2, 1, &m, s);
+                                   kG * (kD + 2), kD + 2, 32 * (kD + 2), 1, &m, s);
   if (ws != KVQ_OK) return ws;
   return launch_merge(m, s);
 }

@@ -274,7 +274,8 @@ kvq_status generic_launch(const AttendArgs& a, cudaStream_t s) {
   m.Lq = a.Lq;
   m.causal = a.causal;
   const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(ctas, a.g.B, a.g.H_kv)),
-                                   static_cast<long long>(n_rt) * kRT * (a.g.D + 2), a.g.D + 2, 1, &m, s);
+                                   static_cast<long long>(n_rt) * kRT * (a.g.D + 2), a.g.D + 2,
+                                   32LL * (a.g.D + 2), 1, &m, s);
   if (ws != KVQ_OK) return ws;
   return launch_merge(m, s);
 }

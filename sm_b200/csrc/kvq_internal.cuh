@@ -111,7 +111,7 @@ __device__ __forceinline__ int seq_blocks(int len, int n_cap, int bt) {
 // Merge partial states of a split (b, h) and write the output rows.
 struct MergeArgs {
   const float* partials;           // row-major: [slots][R_pad][D + 2] : m, z, u[D]
-                                   // feature-major: [slots][D + 2][R_pad]
+                                   // feature-major: [slots][R_pad / 32][D + 2][32]
   const int32_t* lengths;
   void* O;
   int o_dtype;
@@ -131,8 +131,9 @@ kvq_status launch_merge(const MergeArgs& a, cudaStream_t s);
 
 // The window's partial state (m, z, u) of every row of every (b, h), written
 // into slot slot0 + b * H_kv + h of the caller's partial layout: element
-// (row r, field f) of a slot at r * row_stride + f * field_stride (field 0 =
-// m in natural-log units, 1 = z, 2 + d = u[d]).
+// (row r, field f) of a slot at (r / 32) * row_chunk_stride + (r % 32) *
+// row_stride + f * field_stride (field 0 = m in natural-log units, 1 = z,
+// 2 + d = u[d]).
 struct WindowArgs {
   const void* Q;
   int q_dtype;
@@ -144,7 +145,7 @@ struct WindowArgs {
   int B, H_kv, G, Lq, D;
   float scale;
   float* partials;
-  long long slot0, slot_stride, row_stride, field_stride;
+  long long slot0, slot_stride, row_stride, row_chunk_stride, field_stride;
 };
 kvq_status launch_window(const WindowArgs& w, cudaStream_t s);
 
@@ -154,7 +155,8 @@ struct AttendArgs;
 // `partials` (laid out with the given strides, in floats) and point the
 // merge at them.  Without a window it does nothing.
 kvq_status add_window(const AttendArgs& a, float* partials, long long slot0, long long slot_stride,
-                      long long row_stride, long long field_stride, MergeArgs* m, cudaStream_t s);
+                      long long row_stride, long long row_chunk_stride, long long field_stride, MergeArgs* m,
+                      cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // kernels' host launchers

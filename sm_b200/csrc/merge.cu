@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergePara
 
 // Feature-major merge: one CTA per (b, h), 32-row chunk and 32-feature
 // slice; lane = row, so each field read of a part is one coalesced 128-byte
-// line, and warp w owns features 4w .. 4w + 3 of the slice.  A thread loads
+// line, and a chunk's fields are consecutive lines (a slice's 32 features
+// are 4 KB in one run); warp w owns features 4w .. 4w + 3.  A thread loads
 // m, z and its four u values of up to kFmPB parts in one round.
 constexpr int kFmRows = 32;       // rows per CTA
 constexpr int kFmF = 4;           // features per thread
@@ -219,8 +220,8 @@ __global__ void __launch_bounds__(kFmWarps * 32, 3) merge_fm_kernel(MergeParams 
   }
   if (pl.skip || !live) return;
   const long long slot_floats = static_cast<long long>(D + 2) * a.R_pad;
-  const long long rp = a.R_pad;
-  const float* col = a.partials + r;              // part c of this row: col + part_slot(c) * slot_floats
+  // field f of row r within a slot: (r / 32) * (D + 2) * 32 + f * 32 + r % 32
+  const float* col = a.partials + static_cast<long long>(r >> 5) * (D + 2) * 32 + (r & 31);
   float M = -INFINITY, Z = 0.f, U[kFmF];
 #pragma unroll
   for (int j = 0; j < kFmF; ++j) U[j] = 0.f;
@@ -231,9 +232,9 @@ __global__ void __launch_bounds__(kFmWarps * 32, 3) merge_fm_kernel(MergeParams 
       const int c = min(base + k, pl.total - 1);
       const float* part = col + part_slot(pl, c, bh) * slot_floats;
       mc[k] = part[0];
-      zc[k] = part[rp];
+      zc[k] = part[32];
 #pragma unroll
-      for (int j = 0; j < kFmF; ++j) uc[k][j] = j < nf ? part[(2 + f0 + j) * rp] : 0.f;
+      for (int j = 0; j < kFmF; ++j) uc[k][j] = j < nf ? part[(2 + f0 + j) * 32] : 0.f;
     }
     fold_batch<kFmPB, kFmF>(M, Z, U, mc, zc, uc, pl.total - base);
   }
@@ -261,7 +262,7 @@ kvq_status launch_merge(const MergeArgs& a, cudaStream_t s) {
   if (a.feature_major) {
     const int chunks = (a.R + kFmRows - 1) / kFmRows;
     const int slices = (a.D + kFmWarps * kFmF - 1) / (kFmWarps * kFmF);
-    if (chunks > 65535 || slices > 65535 || (a.D % 8) != 0) return KVQ_ERR_UNSUPPORTED;
+    if (chunks > 65535 || slices > 65535 || (a.D % 8) != 0 || (a.R_pad % 32) != 0) return KVQ_ERR_UNSUPPORTED;
     le = launch_pdl(merge_fm_kernel, dim3(static_cast<unsigned>(bh), static_cast<unsigned>(chunks),
                                           static_cast<unsigned>(slices)),
                     dim3(kFmWarps * 32), smem, s, mp);

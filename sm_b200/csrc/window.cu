@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(kWThreads) window_kernel(WindowParams wp) {
     for (int i = threadIdx.x; i < rows * (D + 2); i += blockDim.x) {
       const int r = i / (D + 2), f = i - r * (D + 2);
       const float v = f == 0 ? s_m[r] : (f == 1 ? s_z[r] : s_u[r * D + f - 2]);
-      slot[static_cast<long long>(r0 + r) * a.row_stride + static_cast<long long>(f) * a.field_stride] = v;
+      const long long rr = r0 + r;
+      slot[(rr >> 5) * a.row_chunk_stride + (rr & 31) * a.row_stride + static_cast<long long>(f) * a.field_stride] = v;
     }
     __syncthreads();
   }
@@ -160,7 +161,8 @@ __global__ void __launch_bounds__(kWThreads) window_kernel(WindowParams wp) {
 }  // namespace
 
 kvq_status add_window(const AttendArgs& a, float* partials, long long slot0, long long slot_stride,
-                      long long row_stride, long long field_stride, MergeArgs* m, cudaStream_t s) {
+                      long long row_stride, long long row_chunk_stride, long long field_stride, MergeArgs* m,
+                      cudaStream_t s) {
   if (!a.win_lengths) return KVQ_OK;
   WindowArgs w{};
   w.Q = a.Q;
@@ -180,6 +182,7 @@ kvq_status add_window(const AttendArgs& a, float* partials, long long slot0, lon
   w.slot0 = slot0;
   w.slot_stride = slot_stride;
   w.row_stride = row_stride;
+  w.row_chunk_stride = row_chunk_stride;
   w.field_stride = field_stride;
   const kvq_status st = launch_window(w, s);
   if (st != KVQ_OK) return st;
