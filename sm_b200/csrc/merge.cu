@@ -78,6 +78,26 @@ __device__ __forceinline__ long long part_slot(const MergePlan& p, int i, long l
   return i < p.parts ? p.c_first + i + bh : p.win_slot;
 }
 
+// exp(x) for the merge weights (x <= 0, natural-log units) as one ex2.approx:
+// relative error ~2^-22, far inside the attention tolerance; exp(-inf) = 0.
+__device__ __forceinline__ float exp_w(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  return y;
+}
+
+// The merge plan of the CTA's (b, h), computed by one thread (after warp 0
+// filled s_pre) and shared: its 64-bit divisions run once per CTA.
+__device__ __forceinline__ MergePlan shared_plan(const MergeArgs& a, const int* s_pre, int b, int h,
+                                                 unsigned int* err, bool report, MergePlan* s_plan) {
+  if (threadIdx.x < 32) {
+    __syncwarp();
+    if (threadIdx.x == 0) *s_plan = merge_plan(a, s_pre, b, h, err, report);
+  }
+  __syncthreads();
+  return *s_plan;
+}
+
 // Folds a batch of parts into a running state (M, Z, U[]) with the same
 // rule: the batch's largest m over parts that exist (k < n) and hold a key
 // (z > 0) becomes the reference if it is larger, the state is scaled by
@@ -91,7 +111,7 @@ __device__ __forceinline__ void fold_batch(float& M, float& Z, float (&U)[F], co
   for (int k = 0; k < PB; ++k)
     if (k < n && zc[k] > 0.f) mb = fmaxf(mb, mc[k]);
   if (mb == -INFINITY) return;                       // no key yet
-  const float sa = expf(M - mb);                     // 0 while M = -inf (Z, U are 0)
+  const float sa = exp_w(M - mb);                    // 0 while M = -inf (Z, U are 0)
   Z *= sa;
 #pragma unroll
   for (int j = 0; j < F; ++j) U[j] *= sa;
@@ -99,7 +119,7 @@ __device__ __forceinline__ void fold_batch(float& M, float& Z, float (&U)[F], co
 #pragma unroll
   for (int k = 0; k < PB; ++k) {
     if (k < n && zc[k] > 0.f) {
-      const float w = expf(mc[k] - M);
+      const float w = exp_w(mc[k] - M);
       Z = fmaf(w, zc[k], Z);
 #pragma unroll
       for (int j = 0; j < F; ++j) U[j] = fmaf(w, uc[k][j], U[j]);
@@ -121,9 +141,9 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergePara
   extern __shared__ int s_pre[];                 // [B + 1]
   __shared__ float s_m[kRowMaxWarps], s_z[kRowMaxWarps];
   __shared__ float s_u[kRowMaxWarps][256];
+  __shared__ MergePlan s_plan;
   const MergeArgs& a = mp.a;
   if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
-  __syncthreads();
   const int H = a.H_kv;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
@@ -131,7 +151,7 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergePara
   const int r = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const long long row = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r;
-  const MergePlan pl = merge_plan(a, s_pre, b, h, mp.err, h == 0 && r == 0 && threadIdx.x == 0);
+  const MergePlan pl = shared_plan(a, s_pre, b, h, mp.err, h == 0 && r == 0, &s_plan);
   if (pl.zero) {
     for (int d = threadIdx.x; d < D; d += blockDim.x) store_from_f32(a.O, row * D + d, 0.f, a.o_dtype);
     return;
@@ -176,7 +196,7 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergePara
     float z = 0.f, u = 0.f;
     for (int w = 0; w < nw; ++w) {
       if (s_z[w] > 0.f) {
-        const float e = expf(s_m[w] - Mt);
+        const float e = exp_w(s_m[w] - Mt);
         z = fmaf(e, s_z[w], z);
         u = fmaf(e, s_u[w][d], u);
       }
@@ -198,10 +218,10 @@ constexpr int kFmPB = 8;          // parts per round
 __global__ void __launch_bounds__(kFmWarps * 32, 3) merge_fm_kernel(MergeParams mp) {
   griddep_wait();
   extern __shared__ int s_pre[];                   // [B + 1]
+  __shared__ MergePlan s_plan;
   const MergeArgs& a = mp.a;
   const int D = a.D;
   if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
-  __syncthreads();
   const int H = a.H_kv;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
@@ -209,8 +229,7 @@ __global__ void __launch_bounds__(kFmWarps * 32, 3) merge_fm_kernel(MergeParams 
   const int r = blockIdx.y * kFmRows + lane;
   const int f0 = blockIdx.z * (kFmWarps * kFmF) + kFmF * warp;
   const long long row = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r;
-  const MergePlan pl =
-      merge_plan(a, s_pre, b, h, mp.err, h == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0);
+  const MergePlan pl = shared_plan(a, s_pre, b, h, mp.err, h == 0 && blockIdx.y == 0 && blockIdx.z == 0, &s_plan);
   const bool live = r < a.R && f0 < D;
   const int nf = min(kFmF, D - f0);
   if (pl.zero) {
