@@ -107,20 +107,36 @@ __global__ void __launch_bounds__(kThreads) attend_generic_kernel(GenericParams 
     for (; j < j_end; ++j) {
       const int t_base = j * kBT;
       const int nt = min(kBT, len - t_base);
-      for (int idx = threadIdx.x; idx < kBT * D; idx += blockDim.x) {
-        const int t = idx / D, d = idx - t * D;
-        float kv = 0.f, vv = 0.f;
-        if (t < nt) {
-          const long long tok = t_base + t;
-          const int kcode = code_at(kc, tok * D + d, p.bits);
-          kv = __fmul_rn(static_cast<float>(kcode) - static_cast<float>(qmax),
-                         ks[(tok / p.group) * D + d]);
-          const int vcode = code_at(vc, tok * p.Dp + d, p.bits);
-          vv = __fmul_rn(static_cast<float>(vcode) - static_cast<float>(qmax),
-                         vs[tok * ngv + d / p.group]);
+      // decode the block's K and V into shared memory, kU elements a thread
+      // per round with every load of the round issued before any use
+      constexpr int kU = 4;
+      for (int i0 = 0; i0 < kBT * D; i0 += kU * kThreads) {
+        int kcode[kU], vcode[kU];
+        float ksc[kU], vsc[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int idx = i0 + u * kThreads + static_cast<int>(threadIdx.x);
+          const int t = idx / D, d = idx - t * D;
+          kcode[u] = vcode[u] = 0;
+          ksc[u] = vsc[u] = 0.f;
+          if (idx < kBT * D && t < nt) {
+            const long long tok = t_base + t;
+            kcode[u] = code_at(kc, tok * D + d, p.bits);
+            ksc[u] = ks[(tok / p.group) * D + d];
+            vcode[u] = code_at(vc, tok * p.Dp + d, p.bits);
+            vsc[u] = vs[tok * ngv + d / p.group];
+          }
         }
-        s_k[t * DS + d] = kv;
-        s_v[t * DS + d] = vv;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int idx = i0 + u * kThreads + static_cast<int>(threadIdx.x);
+          if (idx < kBT * D) {
+            const int t = idx / D, d = idx - t * D;
+            const bool in = t < nt;
+            s_k[t * DS + d] = in ? __fmul_rn(static_cast<float>(kcode[u]) - static_cast<float>(qmax), ksc[u]) : 0.f;
+            s_v[t * DS + d] = in ? __fmul_rn(static_cast<float>(vcode[u]) - static_cast<float>(qmax), vsc[u]) : 0.f;
+          }
+        }
       }
       __syncthreads();
       for (int idx = threadIdx.x; idx < kRT * kBT; idx += blockDim.x) {
@@ -136,24 +152,29 @@ __global__ void __launch_bounds__(kThreads) attend_generic_kernel(GenericParams 
         s_p[idx] = sc;
       }
       __syncthreads();
-      if (threadIdx.x < rows) {
-        const int r = threadIdx.x;
-        float mb = -INFINITY;
-        for (int t = 0; t < nt; ++t) mb = fmaxf(mb, s_p[r * kBT + t]);
+      // the block rule per row: a warp per row, lane t = token t (kBT = 32)
+      static_assert(kBT == 32, "one token per lane");
+      for (int r = static_cast<int>(threadIdx.x >> 5); r < rows; r += kThreads / 32) {
+        const int t = static_cast<int>(threadIdx.x & 31);
+        const float sc = t < nt ? s_p[r * kBT + t] : -INFINITY;
+        float mb = sc;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
         const float mo = s_m[r];
         const float mn = fmaxf(mo, mb);
-        const float a = (mo == -INFINITY) ? 0.f : expf(mo - mn);
-        float zs = 0.f;
-        for (int t = 0; t < kBT; ++t) {
-          // a masked key is -inf, and so is mn while a causal row has seen no key
-          const float sc = s_p[r * kBT + t];
-          const float e = (t < nt && sc != -INFINITY) ? expf(sc - mn) : 0.f;
-          s_p[r * kBT + t] = e;
-          zs += e;
+        // a masked key is -inf, and so is mn while a causal row has seen no key
+        const float e = sc != -INFINITY ? expf(sc - mn) : 0.f;
+        s_p[r * kBT + t] = e;
+        float zs = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+        __syncwarp();
+        if (t == 0) {
+          const float a = (mo == -INFINITY) ? 0.f : expf(mo - mn);
+          s_z[r] = a * s_z[r] + zs;
+          s_m[r] = mn;
+          s_a[r] = a;
         }
-        s_z[r] = a * s_z[r] + zs;
-        s_m[r] = mn;
-        s_a[r] = a;
       }
       __syncthreads();
       for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
