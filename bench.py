@@ -262,13 +262,29 @@ def copy_rows_h2d(dst, src, stream) -> None:
     import torch
     global _CUDART
     if "_CUDART" not in globals():
-        import nvidia.cuda_runtime as rt
-        lib = ctypes.CDLL(os.path.join(list(rt.__path__)[0], "lib", "libcudart.so.12"))
-        fn = lib.cudaMemcpy2DAsync
-        fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_size_t,
-                       ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
-        fn.restype = ctypes.c_int
+        fn = None
+        names = []
+        try:
+            import nvidia.cuda_runtime as rt
+            names.append(os.path.join(list(rt.__path__)[0], "lib", "libcudart.so.12"))
+        except ImportError:
+            pass
+        names += ["libcudart.so.12", "libcudart.so"]
+        for name in names:
+            try:
+                fn = ctypes.CDLL(name).cudaMemcpy2DAsync
+                break
+            except (OSError, AttributeError):
+                continue
+        if fn is not None:
+            fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_size_t,
+                           ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+            fn.restype = ctypes.c_int
         _CUDART = fn
+    if _CUDART is None:                     # no runtime library found: torch's copy (a staging kernel)
+        with torch.cuda.stream(stream):
+            dst.copy_(src, non_blocking=True)
+        return
     B_, H_, L_, D_ = src.shape
     assert dst.shape == src.shape and src.is_contiguous() and dst.stride(3) == 1
     assert dst.stride(0) == H_ * dst.stride(1) and dst.stride(2) == D_

@@ -36,3 +36,25 @@ def test_profile_records_exist_and_parse():
     assert bench.recorded_traffic(__file__, "decode_gqa", 4, 32) is None        # hash mismatch
     assert bench.recorded_traffic(__file__, "no_such_workload", 4, 32) is None
     assert bench.recorded_traffic(__file__, "decode_gqa", 4, 32, window=31) is None
+
+
+@__import__("pytest").mark.gpu
+def test_copy_rows_h2d_matches_slice_copy():
+    """The e2e loop's pitched copy of pinned host rows into the last rows of
+    each (b, h) window lands exactly where a slice assignment puts them and
+    leaves the other rows alone."""
+    import pytest
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dev = torch.device("cuda", 0)
+    g = torch.Generator().manual_seed(3)
+    for L in (1, 5):
+        win = torch.randn(3, 4, 32, 128, generator=g).to(dev)
+        want = win.clone()
+        rows = torch.randn(3, 4, L, 128, generator=g).pin_memory()
+        want[:, :, -L:] = rows.to(dev)
+        s = torch.cuda.Stream(dev)
+        bench.copy_rows_h2d(win[:, :, -L:], rows, s)
+        s.synchronize()
+        assert torch.equal(win, want)
