@@ -209,13 +209,15 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergePara
 // slice; lane = row, so each field read of a part is one coalesced 128-byte
 // line, and a chunk's fields are consecutive lines (a slice's 32 features
 // are 4 KB in one run); warp w owns features 4w .. 4w + 3.  A thread loads
-// m, z and its four u values of up to kFmPB parts in one round.
+// m, z and its four u values of kFmPB parts per round; small rounds keep
+// the registers low enough for five CTAs per SM, so the grid runs in fewer
+// waves (each wave pays the prefix and plan chain once).
 constexpr int kFmRows = 32;       // rows per CTA
 constexpr int kFmF = 4;           // features per thread
 constexpr int kFmWarps = 8;       // 8 x 4 = 32 features per CTA
-constexpr int kFmPB = 8;          // parts per round
+constexpr int kFmPB = 4;          // parts per round (two rounds for the usual 5-6)
 
-__global__ void __launch_bounds__(kFmWarps * 32, 3) merge_fm_kernel(MergeParams mp) {
+__global__ void __launch_bounds__(kFmWarps * 32, 5) merge_fm_kernel(MergeParams mp) {
   griddep_wait();
   extern __shared__ int s_pre[];                   // [B + 1]
   __shared__ MergePlan s_plan;
