@@ -135,6 +135,7 @@ PROFILE_FOR = {
     ("decode_gqa", 8, 32): "attend_decode_gqa_b32_ctx4096_8bit.md",
     ("chunk", 4, 32): "attend_chunk_b4_lq64_ctx16384.md",
     ("chunk", 8, 32): "attend_chunk_b4_lq64_ctx16384_8bit.md",
+    ("long_context", 4, 32): "attend_decode_long_b8_ctx1000_32768.md",
 }
 
 
@@ -724,7 +725,9 @@ def study_gqa(K, dev, stream, flush, workload: str, bits: int, n_rep: int = 50):
     med_s = d["median"] * 1e-6
     abytes = attend_bytes(B, H_q, H_kv, D, lens_np, bits, g, lq=Lq)
     flops = 4 * H_q * Lq * D * int(np.sum(lens_np.astype(np.int64)))
+    src = os.path.join(ROOT, "sm_b200", "csrc", "attend_chunk.cu" if Lq > 1 else "attend_decode.cu")
     res = {"attend_us": d, "kernel": K.kernel_name(cache, H_q, Lq), "launches_per_attend": launches,
+           "traffic": recorded_traffic(src, workload, bits, g),
            "bits": bits, "group": g, "B": B, "H_q": H_q, "H_kv": H_kv, "d_h": D, "lq": Lq,
            "lengths_sum": int(np.sum(lens_np)), "algorithmic_bytes": abytes, "flops": flops,
            "gbs": round(abytes / med_s / 1e9, 1)}
