@@ -121,25 +121,25 @@ size_t smem_bytes(int B) { return 1024 + kOffPre + sizeof(int) * (2 * B + 1); }
 // The code - qmax step is exact in f32; the product with the f32 scale is
 // rounded once, to bf16.  Tokens at or past nv become zeros.
 
-// 4-bit: lane = 8 tokens x 4 chunks of 32 features; a byte's two nibbles go
-// into one f32x2 pair (nibble_pair), one FMA makes them n - 7 exactly.  Lane
-// q handles its four words in the order q, q + 1, ... (mod 4): the eight lanes
-// of a quarter warp then store to eight different bank groups, and the K
-// scale loads of a quarter warp hit four groups (lanes of one q share an
-// address).
+// 4-bit: lane = 4 tokens x 8 chunks of 16 features (the 8-bit mapping): a
+// lane's 16 features of a token are one 8-byte code load; a byte's two
+// nibbles go into one f32x2 pair (nibble_pair) and one FMA makes them n - 7
+// exactly.  Lanes q and q + 4 take their two 8-feature halves in opposite
+// order, so a quarter warp (one token) stores to eight different bank groups.
 template <bool kV>
 __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned char* dst, int wk, int lane, int nv) {
   constexpr int kCb = 64;
-  const int q = lane & 3, tt = lane >> 2;
+  const int q = lane & 7, tt = lane >> 3;
+  const bool swap = (q & 4) != 0;
   const float* sc = reinterpret_cast<const float*>(u + kBT * kCb);
-  u64 ks[16];                                   // slot 4 i + r: pair r of word (i + q) mod 4
+  u64 ks[8];                                    // slot 4 i + r: pair r of 8-feature half i ^ swap
   if (!kV) {
     if (16 * wk < nv) {
-      const float4* s4 = reinterpret_cast<const float4*>(sc + (wk >> 1) * kD + 32 * q);
+      const float4* s4 = reinterpret_cast<const float4*>(sc + (wk >> 1) * kD + 16 * q);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int wi = (i + q) & 3;
-        const float4 v0 = s4[2 * wi], v1 = s4[2 * wi + 1];
+      for (int i = 0; i < 2; ++i) {
+        const int ci = i ^ (swap ? 1 : 0);
+        const float4 v0 = s4[2 * ci], v1 = s4[2 * ci + 1];
         ks[4 * i] = pack2(v0.x, v0.y);
         ks[4 * i + 1] = pack2(v0.z, v0.w);
         ks[4 * i + 2] = pack2(v1.x, v1.y);
@@ -147,51 +147,41 @@ __device__ __forceinline__ void decode_unit4(const unsigned char* u, unsigned ch
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) ks[i] = 0ull;
+      for (int i = 0; i < 8; ++i) ks[i] = 0ull;
     }
   }
   const u64 mul = pack2(256.f, 16.f), add = pack2(-263.f, -23.f);
 #pragma unroll 1
-  for (int it = 0; it < 2; ++it) {
-    const int t = 16 * wk + 8 * it + tt;
-    uint4 o[4];
+  for (int it = 0; it < 4; ++it) {
+    const int t = 16 * wk + 4 * it + tt;
+    uint4 o[2];
     if (t < nv) {
-      const uint4 w4 = *reinterpret_cast<const uint4*>(u + t * kCb + 16 * q);
-      // w[i] = word (i + q) mod 4
-      uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-      {
-        const bool c = (q & 2) != 0;
-        const uint32_t x0 = c ? w[2] : w[0], x1 = c ? w[3] : w[1], x2 = c ? w[0] : w[2], x3 = c ? w[1] : w[3];
-        w[0] = x0, w[1] = x1, w[2] = x2, w[3] = x3;
-      }
-      {
-        const bool c = (q & 1) != 0;
-        const uint32_t x0 = c ? w[1] : w[0], x1 = c ? w[2] : w[1], x2 = c ? w[3] : w[2], x3 = c ? w[0] : w[3];
-        w[0] = x0, w[1] = x1, w[2] = x2, w[3] = x3;
-      }
+      const uint2 w2 = *reinterpret_cast<const uint2*>(u + t * kCb + 8 * q);
+      const uint32_t w[2] = {swap ? w2.y : w2.x, swap ? w2.x : w2.y};
       u64 s2 = 0ull;
       if (kV) {
-        const float s = sc[4 * t + q];
+        const float s = sc[4 * t + (q >> 1)];
         s2 = pack2(s, s);
       }
+      uint32_t h[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t h[4];
+      for (int i = 0; i < 2; ++i) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const u64 f = fma2(nibble_pair(byte_at15(w[i], r)), mul, add);
           const u64 x = mul2(f, kV ? s2 : ks[4 * i + r]);
-          h[r] = pack_bf16(lo_f(x), hi_f(x));
+          h[4 * i + r] = pack_bf16(lo_f(x), hi_f(x));
         }
-        o[i] = make_uint4(h[0], h[1], h[2], h[3]);
       }
+      o[0] = make_uint4(h[0], h[1], h[2], h[3]);
+      o[1] = make_uint4(h[4], h[5], h[6], h[7]);
     } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[i] = make_uint4(0u, 0u, 0u, 0u);
+      o[0] = make_uint4(0u, 0u, 0u, 0u);
+      o[1] = o[0];
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int ch = 4 * q + ((i + q) & 3);
+    for (int i = 0; i < 2; ++i) {
+      const int ch = 2 * q + (i ^ (swap ? 1 : 0));
       *reinterpret_cast<uint4*>(dst + (ch >> 3) * kTileHalf + swz(t, ch & 7)) = o[i];
     }
   }
