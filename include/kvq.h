@@ -64,7 +64,7 @@ typedef enum {
   KVQ_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute query) */
   KVQ_ERR_DEVICE = 6,       /* a kernel recorded an internal inconsistency */
   KVQ_ERR_TIMEOUT = 7,      /* a bounded wait inside a kernel ran out */
-  KVQ_ERR_UNSUPPORTED = 8   /* valid arguments outside what this build implements */
+  KVQ_ERR_UNSUPPORTED = 8   /* valid arguments outside what this library implements */
 } kvq_status;
 
 typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;

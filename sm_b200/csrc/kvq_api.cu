@@ -377,7 +377,7 @@ const char* kvq_strerror(kvq_status status) {
     case KVQ_ERR_CUDA: return "CUDA runtime error";
     case KVQ_ERR_DEVICE: return "kernel reported an internal inconsistency";
     case KVQ_ERR_TIMEOUT: return "bounded wait inside a kernel ran out";
-    case KVQ_ERR_UNSUPPORTED: return "arguments outside what this build implements";
+    case KVQ_ERR_UNSUPPORTED: return "arguments outside what this library implements";
   }
   return "unknown status";
 }
