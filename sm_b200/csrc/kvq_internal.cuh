@@ -58,6 +58,20 @@ __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The split form, for a kernel launched right after one that started with
+// griddep_wait() (so every grid before that one has completed by the time this
+// one is scheduled), which reads only the call's inputs and writes workspace
+// that no grid in flight touches: it lets the next kernel be scheduled at once
+// (griddep_release), runs beside its predecessor, and waits for it only at
+// its end (griddep_join), so that its own completion still implies the
+// predecessor's -- the kernel after it reads what both wrote.
+__device__ __forceinline__ void griddep_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_join() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                        Args&&... args) {

@@ -12,113 +12,288 @@
 // kv-block-decode-cost, section "Do not average independently normalized
 // blocks").
 //
-// One CTA per (b, h_kv).  Rows are taken 32 at a time; window tokens 32 at a
-// time are staged in shared memory as f32, their scores computed, and the
-// rows' running (m, z, u) updated with the same rule.  The window is short
-// (a few groups at most), so this is a small kernel next to the packed path.
+// One CTA of eight warps per (b, h_kv, pass), a pass being up to 32 of the
+// head's query rows (RP rows); window tokens 32 at a time are staged in
+// shared memory as f32, their scores computed, and the rows' running
+// (m, z, u) updated with the same rule.  Every index is warp-strided -- warp w owns rows (or tokens)
+// w, w + 8, w + 16, w + 24 and lane l owns features l, l + 32, ... -- so no
+// division runs per element, and a pass's Q rows go out in one batch of loads
+// with the first tile's K and V rows.  The kernel reads only the call's inputs
+// and writes its own slots, so it runs beside the packed-cache kernel before
+// it and joins that kernel's grid only at its end.
 #include "kvq_internal.cuh"
 
 namespace kvq {
 namespace {
 
 constexpr int kWT = 32;          // window tokens per tile
-constexpr int kWR = 32;          // rows per pass
+constexpr int kWR = 32;          // largest rows per pass
 constexpr int kWThreads = 256;
+constexpr int kWWarps = kWThreads / 32;
 static_assert(kWT == 32, "the softmax of a tile runs one token per lane");
+static_assert(kWT == 4 * kWWarps && kWR == 4 * kWWarps, "a warp stages four rows of a tile");
 
 struct WindowParams {
   WindowArgs a;
 };
 
-// shared memory: q [kWR][D], u [kWR][D], K and V tiles [kWT][D + 1],
-// p [kWR][kWT], m, z, alpha [kWR]
-size_t window_smem(int D) {
-  return sizeof(float) * (2 * static_cast<size_t>(kWR) * D + 2 * static_cast<size_t>(kWT) * (D + 1) +
-                          kWR * kWT + 3 * kWR);
+int rows_per_pass(const WindowArgs& a) {
+  const int R = a.G * a.Lq;
+  return R < kWR ? (R < 1 ? 1 : R) : kWR;
 }
 
-__global__ void __launch_bounds__(kWThreads) window_kernel(WindowParams wp) {
-  griddep_wait();
+// shared memory: q [RP][D], u [RP][D], K and V tiles [kWT][D + 1],
+// p [RP][kWT], m, z, alpha [RP]
+size_t window_smem(int D, int RP) {
+  return sizeof(float) * (2 * static_cast<size_t>(RP) * D + 2 * static_cast<size_t>(kWT) * (D + 1) +
+                          static_cast<size_t>(RP) * kWT + 3 * static_cast<size_t>(RP));
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// rows warp + 8k (k < 4) of the row-major [.][D] array at p, feature
+// lane + 32j in v[k][j]; rows at or past n_live and features past D read 0
+template <int JMAX, typename T>
+__device__ __forceinline__ void load_rows(float (&v)[4][JMAX], const T* p, int D, int n_live, int warp, int lane) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = warp + kWWarps * k;
+#pragma unroll
+    for (int j = 0; j < JMAX; ++j) {
+      const int d = lane + 32 * j;
+      v[k][j] = (r < n_live && d < D) ? to_f32(p[static_cast<long long>(r) * D + d]) : 0.f;
+    }
+  }
+}
+
+template <int JMAX>
+__device__ __forceinline__ void load_rows_any(float (&v)[4][JMAX], const void* p, int dtype, long long off, int D,
+                                              int n_live, int warp, int lane) {
+  if (dtype == KVQ_F32) load_rows<JMAX>(v, static_cast<const float*>(p) + off, D, n_live, warp, lane);
+  else load_rows<JMAX>(v, static_cast<const __nv_bfloat16*>(p) + off, D, n_live, warp, lane);
+}
+
+// v[k][j] to s[(warp + 8k) * stride + lane + 32j] for the rows below n_rows
+template <int JMAX>
+__device__ __forceinline__ void store_rows(float* s, int stride, const float (&v)[4][JMAX], int D, int n_rows,
+                                           int warp, int lane) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = warp + kWWarps * k;
+#pragma unroll
+    for (int j = 0; j < JMAX; ++j) {
+      const int d = lane + 32 * j;
+      if (r < n_rows && d < D) s[r * stride + d] = v[k][j];
+    }
+  }
+}
+
+// Scores of a tile, s_p[r][t] = scale * q_r . k_t, for a pass of at most 8
+// rows: item (r, t) per thread; when there are fewer items than threads,
+// `parts` adjacent lanes split an item's dot product (features part, part +
+// parts, ...) and add with shuffles.
+__device__ __forceinline__ void scores_few_rows(float* s_p, const float* s_q, const float* s_k, int rows, int nt,
+                                                int D, int DS, float scale) {
+  const int items = rows * kWT;
+  const int parts = items * 2 > kWThreads ? 1 : items * 4 > kWThreads ? 2 : items * 8 > kWThreads ? 4 : 8;
+  const int per = kWThreads / parts;                 // items per sweep
+  for (int base = 0; base < items; base += per) {
+    const int it = base + static_cast<int>(threadIdx.x) / parts;
+    const int pt = static_cast<int>(threadIdx.x) % parts;
+    const int r = it / kWT, t = it - r * kWT;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (it < items && t < nt) {
+      const float* qr = s_q + r * D;
+      const float* kr = s_k + t * DS;
+      int d = pt;
+      for (; d + 3 * parts < D; d += 4 * parts) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = fmaf(qr[d + j * parts], kr[d + j * parts], acc[j]);
+      }
+      for (; d < D; d += parts) acc[0] = fmaf(qr[d], kr[d], acc[0]);
+    }
+    float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    for (int o = 1; o < parts; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (it < items && pt == 0) s_p[r * kWT + t] = t < nt ? sum * scale : -INFINITY;
+  }
+}
+
+// The same for a pass of more rows: warp w takes rows 4w .. 4w + 3, lane l
+// token l, so a K element read once serves four rows (the Q elements are
+// broadcast reads, four features at a time when D is a multiple of 4).
+__device__ __forceinline__ void scores_many_rows(float* s_p, const float* s_q, const float* s_k, int rows, int nt,
+                                                 int D, int DS, float scale, int warp, int lane) {
+  const int rb = 4 * warp;
+  if (rb >= rows) return;
+  const float* q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q[i] = s_q + min(rb + i, rows - 1) * D;
+  const float* kr = s_k + lane * DS;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int d = 0;
+  if ((D & 3) == 0) {
+    for (; d < D; d += 4) {
+      const float k0 = kr[d], k1 = kr[d + 1], k2 = kr[d + 2], k3 = kr[d + 3];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 qv = *reinterpret_cast<const float4*>(q[i] + d);
+        acc[i] = fmaf(qv.x, k0, acc[i]);
+        acc[i] = fmaf(qv.y, k1, acc[i]);
+        acc[i] = fmaf(qv.z, k2, acc[i]);
+        acc[i] = fmaf(qv.w, k3, acc[i]);
+      }
+    }
+  }
+  for (; d < D; ++d) {
+    const float kv = kr[d];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = fmaf(q[i][d], kv, acc[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (rb + i < rows) s_p[(rb + i) * kWT + lane] = lane < nt ? acc[i] * scale : -INFINITY;
+}
+
+// u = alpha u + p V over the tile's tokens (the first tile starts u from
+// zero), for a pass of at most 8 rows: a warp per (row, 32 features), four
+// chains over the tokens.
+__device__ __forceinline__ void pv_few_rows(float* s_u, const float* s_p, const float* s_v, const float* s_a,
+                                            bool first, int rows, int nt, int D, int DS, int warp, int lane) {
+  const int nj = (D + 31) >> 5;
+  for (int item = warp; item < rows * nj; item += kWWarps) {
+    const int r = item / nj, j = item - r * nj;
+    const int d = lane + 32 * j;
+    if (d < D) {
+      const float* pr = s_p + r * kWT;
+      const float* vc = s_v + d;
+      float c0 = first ? 0.f : s_a[r] * s_u[r * D + d], c1 = 0.f, c2 = 0.f, c3 = 0.f;
+      int t = 0;
+      for (; t + 4 <= nt; t += 4) {
+        c0 = fmaf(pr[t], vc[t * DS], c0);
+        c1 = fmaf(pr[t + 1], vc[(t + 1) * DS], c1);
+        c2 = fmaf(pr[t + 2], vc[(t + 2) * DS], c2);
+        c3 = fmaf(pr[t + 3], vc[(t + 3) * DS], c3);
+      }
+      for (; t < nt; ++t) c0 = fmaf(pr[t], vc[t * DS], c0);
+      s_u[r * D + d] = (c0 + c1) + (c2 + c3);
+    }
+  }
+}
+
+// The same for a pass of more rows: warp w takes rows 4w .. 4w + 3, lane l
+// features l, l + 32, ..., so a V element read once serves four rows.
+template <int JMAX>
+__device__ __forceinline__ void pv_many_rows(float* s_u, const float* s_p, const float* s_v, const float* s_a,
+                                             bool first, int rows, int nt, int D, int DS, int warp, int lane) {
+  const int rb = 4 * warp;
+  if (rb >= rows) return;
+  float acc[4][JMAX];
+  int pr[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pr[i] = min(rb + i, rows - 1);
+    const float al = first ? 0.f : s_a[pr[i]];
+#pragma unroll
+    for (int j = 0; j < JMAX; ++j) {
+      const int d = lane + 32 * j;
+      acc[i][j] = (first || d >= D) ? 0.f : al * s_u[pr[i] * D + d];
+    }
+  }
+  for (int t = 0; t < nt; ++t) {
+    float p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = s_p[pr[i] * kWT + t];
+#pragma unroll
+    for (int j = 0; j < JMAX; ++j) {
+      const int d = lane + 32 * j;
+      const float v = s_v[t * DS + min(d, D)];      // column D is the row's padding
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(p[i], v, acc[i][j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < JMAX; ++j) {
+      const int d = lane + 32 * j;
+      if (rb + i < rows && d < D) s_u[(rb + i) * D + d] = acc[i][j];
+    }
+}
+
+// JMAX: features per lane, D <= 32 * JMAX.  One CTA per (b, h_kv, pass of
+// RP rows); the body is a grid-stride loop over the passes, which at this
+// grid runs once (the loop form measured 4 to 8 us faster per step than the
+// same body without it on the decode workload's window).  Two CTAs per SM:
+// the grid of a decode step, B * H_kv CTAs, then fits in one wave.
+template <int JMAX>
+__global__ void __launch_bounds__(kWThreads, 2) window_kernel(WindowParams wp) {
+  griddep_release();
   const WindowArgs& a = wp.a;
   extern __shared__ float sm[];
   const int D = a.D, DS = D + 1;
-  float* s_q = sm;                       // [kWR][D]
-  float* s_u = s_q + kWR * D;            // [kWR][D]
-  float* s_k = s_u + kWR * D;            // [kWT][DS]
-  float* s_v = s_k + kWT * DS;           // [kWT][DS]
-  float* s_p = s_v + kWT * DS;           // [kWR][kWT]
-  float* s_m = s_p + kWR * kWT;
-  float* s_z = s_m + kWR;
-  float* s_a = s_z + kWR;
-
-  const int bh = blockIdx.x;
-  const int b = bh / a.H_kv, h = bh % a.H_kv;
   const int R = a.G * a.Lq;
+  const int RP = R < kWR ? R : kWR;
+  if (RP < 1) {
+    griddep_join();
+    return;
+  }
+  const int passes = (R + RP - 1) / RP;
+  float* s_q = sm;                       // [RP][D]
+  float* s_u = s_q + RP * D;             // [RP][D]
+  float* s_k = s_u + RP * D;             // [kWT][DS]
+  float* s_v = s_k + kWT * DS;           // [kWT][DS]
+  float* s_p = s_v + kWT * DS;           // [RP][kWT]
+  float* s_m = s_p + RP * kWT;
+  float* s_z = s_m + RP;
+  float* s_a = s_z + RP;
+
+  const int bh = static_cast<int>(blockIdx.x) / passes;
+  const int r_first = (static_cast<int>(blockIdx.x) - bh * passes) * RP;
+  const int b = bh / a.H_kv, h = bh % a.H_kv;
   const int raw = a.win_lengths[b];
   const int wl = raw < 0 ? 0 : (raw > a.W_cap ? a.W_cap : raw);
   const long long row_base = (static_cast<long long>(b) * a.H_kv * a.G + static_cast<long long>(h) * a.G) * a.Lq;
   const long long win_base = static_cast<long long>(bh) * a.W_cap * D;
   float* slot = a.partials + (a.slot0 + bh) * a.slot_stride;
-
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int r0 = 0; r0 < R; r0 += kWR) {
-    const int rows = min(kWR, R - r0);
-    for (int i0 = threadIdx.x; i0 < rows * D; i0 += kWThreads * 8) {
-      float qv[8];                                     // eight loads in flight per thread
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * kWThreads;
-        qv[u] = i < rows * D ? load_as_f32(a.Q, (row_base + r0) * D + i, a.q_dtype) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (i0 + u * kWThreads < rows * D) s_q[i0 + u * kWThreads] = qv[u];
+  for (int r0 = r_first; r0 < R; r0 += RP * passes) {
+    const int rows = min(RP, R - r0);
+    const bool many = rows > 8;
+    {
+      // the pass's Q rows and the window's first tile, all loads issued
+      // before any store
+      float qv[4][JMAX], kv[4][JMAX], vv[4][JMAX];
+      const int nt0 = min(kWT, wl);
+      load_rows_any<JMAX>(qv, a.Q, a.q_dtype, (row_base + r0) * D, D, rows, warp, lane);
+      load_rows_any<JMAX>(kv, a.K_win, a.win_dtype, win_base, D, nt0, warp, lane);
+      load_rows_any<JMAX>(vv, a.V_win, a.win_dtype, win_base, D, nt0, warp, lane);
+      store_rows<JMAX>(s_q, D, qv, D, rows, warp, lane);
+      store_rows<JMAX>(s_k, DS, kv, D, kWT, warp, lane);
+      store_rows<JMAX>(s_v, DS, vv, D, kWT, warp, lane);
     }
-    for (int i = threadIdx.x; i < kWR * D; i += blockDim.x) s_u[i] = 0.f;
-    if (threadIdx.x < kWR) {
+    if (threadIdx.x < RP) {
       s_m[threadIdx.x] = -INFINITY;
       s_z[threadIdx.x] = 0.f;
     }
     __syncthreads();
     for (int t0 = 0; t0 < wl; t0 += kWT) {
       const int nt = min(kWT, wl - t0);
-      // the tile's K and V rows, all of a thread's loads issued before any store
-      for (int i0 = threadIdx.x; i0 < kWT * D; i0 += kWThreads * 8) {
-        float kv[8], vv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = i0 + u * kWThreads;
-          const bool live = i < nt * D;
-          const long long e = win_base + static_cast<long long>(t0) * D + i;
-          kv[u] = live ? load_as_f32(a.K_win, e, a.win_dtype) : 0.f;
-          vv[u] = live ? load_as_f32(a.V_win, e, a.win_dtype) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = i0 + u * kWThreads;
-          if (i < kWT * D) {
-            const int t = i / D, d = i - t * D;
-            s_k[t * DS + d] = kv[u];
-            s_v[t * DS + d] = vv[u];
-          }
-        }
+      if (t0 > 0) {
+        float kv[4][JMAX], vv[4][JMAX];
+        const long long off = win_base + static_cast<long long>(t0) * D;
+        load_rows_any<JMAX>(kv, a.K_win, a.win_dtype, off, D, nt, warp, lane);
+        load_rows_any<JMAX>(vv, a.V_win, a.win_dtype, off, D, nt, warp, lane);
+        store_rows<JMAX>(s_k, DS, kv, D, kWT, warp, lane);
+        store_rows<JMAX>(s_v, DS, vv, D, kWT, warp, lane);
+        __syncthreads();
       }
-      __syncthreads();
-      // scores of the tile
-      for (int i = threadIdx.x; i < kWR * kWT; i += blockDim.x) {
-        const int r = i / kWT, t = i - r * kWT;
-        float sc = -INFINITY;
-        if (r < rows && t < nt) {
-          float acc = 0.f;
-          for (int d = 0; d < D; ++d) acc = fmaf(s_q[r * D + d], s_k[t * DS + d], acc);
-          sc = acc * a.scale;
-        }
-        s_p[i] = sc;
-      }
+      if (many) scores_many_rows(s_p, s_q, s_k, rows, nt, D, DS, a.scale, warp, lane);
+      else scores_few_rows(s_p, s_q, s_k, rows, nt, D, DS, a.scale);
       __syncthreads();
       // the block rule: m_new = max(m, tile max), alpha = exp(m - m_new);
       // a warp per row, lane = token of the tile
-      for (int r = warp; r < rows; r += kWThreads / 32) {
+      for (int r = warp; r < rows; r += kWWarps) {
         const float sc = s_p[r * kWT + lane];          // -inf past the tile's tokens
         float mb = sc;
 #pragma unroll
@@ -139,23 +314,22 @@ __global__ void __launch_bounds__(kWThreads) window_kernel(WindowParams wp) {
         }
       }
       __syncthreads();
-      for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
-        const int r = i / D, d = i - r * D;
-        float acc = s_a[r] * s_u[i];
-        for (int t = 0; t < nt; ++t) acc = fmaf(s_p[r * kWT + t], s_v[t * DS + d], acc);
-        s_u[i] = acc;
-      }
+      if (many) pv_many_rows<JMAX>(s_u, s_p, s_v, s_a, t0 == 0, rows, nt, D, DS, warp, lane);
+      else pv_few_rows(s_u, s_p, s_v, s_a, t0 == 0, rows, nt, D, DS, warp, lane);
       __syncthreads();
     }
-    // the rows' window states; an empty window leaves m = -inf, z = 0
-    for (int i = threadIdx.x; i < rows * (D + 2); i += blockDim.x) {
-      const int r = i / (D + 2), f = i - r * (D + 2);
-      const float v = f == 0 ? s_m[r] : (f == 1 ? s_z[r] : s_u[r * D + f - 2]);
+    // the rows' window states; an empty window leaves m = -inf, z = 0, u = 0
+    for (int r = warp; r < rows; r += kWWarps) {
       const long long rr = r0 + r;
-      slot[(rr >> 5) * a.row_chunk_stride + (rr & 31) * a.row_stride + static_cast<long long>(f) * a.field_stride] = v;
+      float* dst = slot + (rr >> 5) * a.row_chunk_stride + (rr & 31) * a.row_stride;
+      for (int f = lane; f < D + 2; f += 32) {
+        const float v = f == 0 ? s_m[r] : (f == 1 ? s_z[r] : (wl > 0 ? s_u[r * D + f - 2] : 0.f));
+        dst[static_cast<long long>(f) * a.field_stride] = v;
+      }
     }
     __syncthreads();
   }
+  griddep_join();
 }
 
 }  // namespace
@@ -193,12 +367,15 @@ kvq_status add_window(const AttendArgs& a, float* partials, long long slot0, lon
 }
 
 kvq_status launch_window(const WindowArgs& w, cudaStream_t s) {
-  const long long blocks = static_cast<long long>(w.B) * w.H_kv;
+  const int RP = rows_per_pass(w);
+  const long long passes = (static_cast<long long>(w.G) * w.Lq + RP - 1) / RP;
+  const long long blocks = static_cast<long long>(w.B) * w.H_kv * (passes < 1 ? 1 : passes);
   if (blocks > 0x7fffffffLL || w.D > 256 || w.D < 1) return KVQ_ERR_UNSUPPORTED;
-  const size_t smem = window_smem(w.D);
-  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(window_kernel), smem)) return KVQ_ERR_CUDA;
+  const size_t smem = window_smem(w.D, RP);
+  auto kernel = w.D <= 64 ? window_kernel<2> : (w.D <= 128 ? window_kernel<4> : window_kernel<8>);
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kernel), smem)) return KVQ_ERR_CUDA;
   WindowParams p{w};
-  if (launch_pdl(window_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kWThreads), smem, s, p) != cudaSuccess)
+  if (launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kWThreads), smem, s, p) != cudaSuccess)
     return KVQ_ERR_CUDA;
   count_launch();
   return KVQ_OK;

@@ -459,6 +459,16 @@ def test_window_generic(sm, bits, group):
     _check_window(sm, q, k, v, lens, kw, vw, wl, bits, group, 0.125, q_dtype=torch.float32)
 
 
+@pytest.mark.parametrize("d", [50, 72])
+def test_window_many_rows(sm, d):
+    """A window pass of more than eight query rows that is not a multiple of
+    four (fourteen: two heads per KV head, seven queries), a head dimension
+    that is not a multiple of 32 (and, at 50, not of 4), two window tiles."""
+    q, k, v, lens = _gqa_case(2, 4, 2, 200, d, [200, 61], lq=7, seed=90 + d)
+    kw, vw, wl = _window(2, 2, 40, d, [40, 9], seed=91 + d)
+    _check_window(sm, q, k, v, lens, kw, vw, wl, 4, 32, 0.125, win_dtype=torch.bfloat16)
+
+
 def test_window_bad_lengths(sm):
     """No key at all (both lengths 0) or a window length past its capacity is
     reported; the keyless sequence's rows are zeros, the others stay finite."""
