@@ -52,7 +52,13 @@ bool make_geometry(const kvq_cache* c, Geometry* g);
 // with griddep_wait() -- which returns once every earlier grid on the stream
 // has completed and its memory is visible -- before any global-memory
 // access; it then lets the next kernel be scheduled.  Without a predecessor
-// (or without the launch attribute) both are no-ops.
+// (or without the launch attribute) both are no-ops.  Two kernels always run
+// right after one of the library's own, which has waited for every grid
+// before it by the time it lets them be scheduled, and read some of the
+// call's inputs (which no kernel of the library writes) before their own
+// wait, through the L2 (ld.global.cg): the split merge computes its plan
+// from the lengths, and the window kernel (griddep_release / griddep_join
+// below) does all its work.
 __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -46,12 +46,12 @@ struct MergePlan {
 __device__ __forceinline__ MergePlan merge_plan(const MergeArgs& a, const int* s_pre, int b, int h,
                                                 unsigned int* err, bool report) {
   const int H = a.H_kv;
-  const int raw = a.lengths[b];
+  const int raw = __ldcg(a.lengths + b);
   const int nb = s_pre[b + 1] - s_pre[b];
   int wl = 0;
   bool bad;
   if (a.win_lengths) {
-    const int wr = a.win_lengths[b];
+    const int wr = __ldcg(a.win_lengths + b);
     wl = wr < 0 ? 0 : (wr > a.W_cap ? a.W_cap : wr);
     bad = raw < 0 || raw > a.N_cap || wr < 0 || wr > a.W_cap || (nb == 0 && wl == 0);
   } else {
@@ -137,13 +137,12 @@ constexpr int kRowF = 8;          // features per lane
 constexpr int kRowMaxWarps = 8;
 
 __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergeParams mp) {
-  griddep_wait();
   extern __shared__ int s_pre[];                 // [B + 1]
   __shared__ float s_m[kRowMaxWarps], s_z[kRowMaxWarps];
   __shared__ float s_u[kRowMaxWarps][256];
   __shared__ MergePlan s_plan;
   const MergeArgs& a = mp.a;
-  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
+  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre, true);
   const int H = a.H_kv;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
@@ -152,6 +151,7 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergePara
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const long long row = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r;
   const MergePlan pl = shared_plan(a, s_pre, b, h, mp.err, h == 0 && r == 0, &s_plan);
+  griddep_wait();                                // the plan ran beside the kernel before; now its parts
   if (pl.zero) {
     for (int d = threadIdx.x; d < D; d += blockDim.x) store_from_f32(a.O, row * D + d, 0.f, a.o_dtype);
     return;
@@ -218,12 +218,11 @@ constexpr int kFmWarps = 8;       // 8 x 4 = 32 features per CTA
 constexpr int kFmPB = 4;          // parts per round (two rounds for the usual 5-6)
 
 __global__ void __launch_bounds__(kFmWarps * 32, 5) merge_fm_kernel(MergeParams mp) {
-  griddep_wait();
   extern __shared__ int s_pre[];                   // [B + 1]
   __shared__ MergePlan s_plan;
   const MergeArgs& a = mp.a;
   const int D = a.D;
-  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre);
+  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre, true);
   const int H = a.H_kv;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
@@ -232,6 +231,7 @@ __global__ void __launch_bounds__(kFmWarps * 32, 5) merge_fm_kernel(MergeParams 
   const int f0 = blockIdx.z * (kFmWarps * kFmF) + kFmF * warp;
   const long long row = (static_cast<long long>(b) * H * a.G + static_cast<long long>(h) * a.G) * a.Lq + r;
   const MergePlan pl = shared_plan(a, s_pre, b, h, mp.err, h == 0 && blockIdx.y == 0 && blockIdx.z == 0, &s_plan);
+  griddep_wait();                                  // the plan ran beside the kernel before; now its parts
   const bool live = r < a.R && f0 < D;
   const int nf = min(kFmF, D - f0);
   if (pl.zero) {

@@ -14,13 +14,15 @@
 namespace kvq {
 
 // Warp 0 fills pre[0..B] (the caller synchronises the CTA afterwards).
+// l2: read the lengths at the L2 (ld.global.cg), as a kernel does that reads
+// them before its grid-dependency wait.
 __device__ __forceinline__ void warp_block_prefix(const int32_t* lengths, int B, int n_cap, int bt,
-                                                  int* pre) {
+                                                  int* pre, bool l2 = false) {
   const int lane = threadIdx.x & 31;
   int carry = 0;
   for (int base = 0; base < B; base += 32) {
     const int b = base + lane;
-    int v = b < B ? seq_blocks(__ldg(lengths + b), n_cap, bt) : 0;
+    int v = b < B ? seq_blocks(l2 ? __ldcg(lengths + b) : __ldg(lengths + b), n_cap, bt) : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int n = __shfl_up_sync(0xffffffffu, v, o);

@@ -53,7 +53,9 @@ __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // rows warp + 8k (k < 4) of the row-major [.][D] array at p, feature
-// lane + 32j in v[k][j]; rows at or past n_live and features past D read 0
+// lane + 32j in v[k][j]; rows at or past n_live and features past D read 0.
+// The reads go to the L2 (ld.global.cg): the kernel reads its inputs before
+// its grid-dependency wait.
 template <int JMAX, typename T>
 __device__ __forceinline__ void load_rows(float (&v)[4][JMAX], const T* p, int D, int n_live, int warp, int lane) {
 #pragma unroll
@@ -62,7 +64,7 @@ __device__ __forceinline__ void load_rows(float (&v)[4][JMAX], const T* p, int D
 #pragma unroll
     for (int j = 0; j < JMAX; ++j) {
       const int d = lane + 32 * j;
-      v[k][j] = (r < n_live && d < D) ? to_f32(p[static_cast<long long>(r) * D + d]) : 0.f;
+      v[k][j] = (r < n_live && d < D) ? to_f32(__ldcg(p + static_cast<long long>(r) * D + d)) : 0.f;
     }
   }
 }
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kWThreads, 2) window_kernel(WindowParams wp) {
   const int bh = static_cast<int>(blockIdx.x) / passes;
   const int r_first = (static_cast<int>(blockIdx.x) - bh * passes) * RP;
   const int b = bh / a.H_kv, h = bh % a.H_kv;
-  const int raw = a.win_lengths[b];
+  const int raw = __ldcg(a.win_lengths + b);
   const int wl = raw < 0 ? 0 : (raw > a.W_cap ? a.W_cap : raw);
   const long long row_base = (static_cast<long long>(b) * a.H_kv * a.G + static_cast<long long>(h) * a.G) * a.Lq;
   const long long win_base = static_cast<long long>(bh) * a.W_cap * D;
