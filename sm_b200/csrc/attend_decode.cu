@@ -400,13 +400,29 @@ __device__ __forceinline__ int part_index(int t, int i) { return t * 32 + ((i ^ 
 // ---------------------------------------------------------------------------
 // iteration over a worker's block range
 // ---------------------------------------------------------------------------
+// A segment is the part of one head that a worker's range covers: plan
+// slots [jb, jb + span) of the head's nb, at global slot gpos, and its blocks
+// [jb, je).  The blocks stop at the head's last block: the decode step's
+// plan has one more slot per head (its append, warp_block_prefix's extra),
+// which holds no block, so a segment can hold that slot alone (jb == je).
 struct Seg {
   int b, h, nb, jb, je;
-  long long gpos;                     // global index of block jb
+  long long gpos;                     // global index of slot jb
   bool valid;
 };
 
-__device__ __forceinline__ Seg first_seg(const int* pre, int B, int H, const CtaRange& cr) {
+// Blocks of a sequence of clamped length len.
+__device__ __forceinline__ int real_blocks(int len) { return (len + kTB - 1) / kTB; }
+
+// SLOT: the decode step's plan with the append slot; without it a head's
+// slots are its blocks.
+template <bool SLOT>
+__device__ __forceinline__ int seg_blocks(const Seg& s, const int* slen) {
+  return SLOT ? real_blocks(slen[s.b]) : s.nb;
+}
+
+template <bool SLOT>
+__device__ __forceinline__ Seg first_seg(const int* pre, const int* slen, int B, int H, const CtaRange& cr) {
   Seg s;
   s.valid = cr.g0 < cr.g1;
   if (!s.valid) return s;
@@ -415,13 +431,15 @@ __device__ __forceinline__ Seg first_seg(const int* pre, int B, int H, const Cta
   const long long off = cr.g0 - static_cast<long long>(H) * pre[s.b];
   s.h = static_cast<int>(off / s.nb);
   s.jb = static_cast<int>(off % s.nb);
-  s.je = static_cast<int>(min(static_cast<long long>(s.nb), s.jb + (cr.g1 - cr.g0)));
+  s.je = static_cast<int>(min(static_cast<long long>(seg_blocks<SLOT>(s, slen)), s.jb + (cr.g1 - cr.g0)));
   s.gpos = cr.g0;
   return s;
 }
 
-__device__ __forceinline__ Seg next_seg(Seg s, const int* pre, int B, int H, const CtaRange& cr) {
-  s.gpos += s.je - s.jb;
+template <bool SLOT>
+__device__ __forceinline__ Seg next_seg(Seg s, const int* pre, const int* slen, int B, int H, const CtaRange& cr) {
+  // past the segment's slots (its blocks, and the append slot if it holds it)
+  s.gpos += SLOT ? min(static_cast<long long>(s.nb), s.jb + (cr.g1 - s.gpos)) - s.jb : s.je - s.jb;
   if (s.gpos >= cr.g1) {
     s.valid = false;
     return s;
@@ -433,7 +451,7 @@ __device__ __forceinline__ Seg next_seg(Seg s, const int* pre, int B, int H, con
   }
   s.nb = pre[s.b + 1] - pre[s.b];
   s.jb = 0;
-  s.je = static_cast<int>(min(static_cast<long long>(s.nb), cr.g1 - s.gpos));
+  s.je = static_cast<int>(min(static_cast<long long>(seg_blocks<SLOT>(s, slen)), cr.g1 - s.gpos));
   return s;
 }
 
@@ -443,9 +461,11 @@ struct Prod {
   bool valid;
 };
 
-__device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, int B, int H, const CtaRange& cr) {
+template <bool SLOT>
+__device__ __forceinline__ Prod prod_settle(Prod p, const int* pre, const int* slen, int B, int H,
+                                            const CtaRange& cr) {
   while (p.valid && p.j >= p.seg.je) {
-    p.seg = next_seg(p.seg, pre, B, H, cr);
+    p.seg = next_seg<SLOT>(p.seg, pre, slen, B, H, cr);
     p.valid = p.seg.valid;
     p.j = p.seg.jb;
   }
@@ -519,9 +539,14 @@ __device__ __forceinline__ void append_tail(const DecodeParams& p, int b, int h,
   const int j = t / GRP, nin = t % GRP + 1;
   const int c = 2 * pt;
   // the group's rows of channels c, c + 1; the dtype branch sits outside the
-  // row loop so the 2 GRP loads go out back to back (one round trip)
-  float x0[GRP], x1[GRP];
+  // row loop so the 2 GRP loads go out back to back (one round trip).  At 4
+  // bits the new V row's two channels go out in the same batch: the worker
+  // that appends covers one block fewer (the plan's append slot), which
+  // leaves it off the tail only if the append costs one round trip (at 8
+  // bits, without the slot, the batched form measured slower)
+  float x0[GRP], x1[GRP], v0 = 0.f, v1 = 0.f;
   const long long e0 = head * GRP * kD + c;
+  const long long ve = head * kD + c;
   if (p.in_dtype == KVQ_F32) {
     const float* src = static_cast<const float*>(p.k_tail) + e0;
 #pragma unroll
@@ -529,12 +554,20 @@ __device__ __forceinline__ void append_tail(const DecodeParams& p, int b, int h,
       x0[r] = r < nin ? src[r * kD] : 0.f;
       x1[r] = r < nin ? src[r * kD + 1] : 0.f;
     }
+    if (BITS == 4) {
+      v0 = static_cast<const float*>(p.v_new)[ve];
+      v1 = static_cast<const float*>(p.v_new)[ve + 1];
+    }
   } else {
     const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.k_tail) + e0;
 #pragma unroll
     for (int r = 0; r < GRP; ++r) {
       x0[r] = r < nin ? __bfloat162float(src[r * kD]) : 0.f;
       x1[r] = r < nin ? __bfloat162float(src[r * kD + 1]) : 0.f;
+    }
+    if (BITS == 4) {
+      v0 = __bfloat162float(static_cast<const __nv_bfloat16*>(p.v_new)[ve]);
+      v1 = __bfloat162float(static_cast<const __nv_bfloat16*>(p.v_new)[ve + 1]);
     }
   }
   float a0 = 0.f, a1 = 0.f;
@@ -556,8 +589,10 @@ __device__ __forceinline__ void append_tail(const DecodeParams& p, int b, int h,
     else *reinterpret_cast<uint16_t*>(kc + row * 128 + c) = static_cast<uint16_t>(q0 | (q1 << 8));
   }
   // V row t: the GRP / 2 threads of a V group (within one warp) share its max
-  const long long ve = head * kD + c;
-  const float v0 = load_as_f32(p.v_new, ve, p.in_dtype), v1 = load_as_f32(p.v_new, ve + 1, p.in_dtype);
+  if (BITS != 4) {
+    v0 = load_as_f32(p.v_new, ve, p.in_dtype);
+    v1 = load_as_f32(p.v_new, ve + 1, p.in_dtype);
+  }
   float am = fmaxf(fabsf(v0), fabsf(v1));
 #pragma unroll
   for (int o = 1; o < GRP / 2; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
@@ -578,6 +613,13 @@ __device__ __forceinline__ void append_tail(const DecodeParams& p, int b, int h,
 template <int BITS, int GRP, bool APPEND>
 __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasPerSm) decode_kernel(DecodeParams p) {
   griddep_wait();
+  // the append slot in the plan (Seg): 4-bit codes only, whose 1,184 workers
+  // leave the split room for it at the decode workload's size (32,768 blocks
+  // and 256 slots in ranges of 28).  Where there is no room (8-bit: 888
+  // workers, ranges of 37 that the slots would make 38) every range grows by
+  // one slot, so 8-bit keeps the plain plan; a runtime choice between the two
+  // measured slower than either at 4 bits.
+  constexpr bool kSlot = APPEND && BITS == 4;
   constexpr int kNP = Tr<BITS, GRP>::kNP, kS = Tr<BITS, GRP>::kS, kThreads = Tr<BITS, GRP>::kThreads;
   using PairSmem = kvq::PairSmem<BITS, GRP>;
   using Stage = kvq::Stage<BITS, GRP>;
@@ -592,7 +634,9 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
   const int ts = lane >> 3, cs = lane & 7;
   PairSmem& ps = pairs[pair];
 
-  if (warp == 0) warp_block_prefix(p.lengths, p.B, p.N_cap, kTB, pre);
+  // the decode step counts its append as one more plan slot per head (Seg):
+  // the workers that append cover one block fewer
+  if (warp == 0) warp_block_prefix(p.lengths, p.B, p.N_cap, kTB, pre, false, kSlot ? 1 : 0);
   for (int b = threadIdx.x; b < p.B; b += kThreads) slen[b] = clamp_len(p.lengths[b], p.N_cap);
   if (is_s && lane == 0) {
 #pragma unroll
@@ -619,14 +663,15 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
   const CtaRange cr = cta_range(pre, p.B, H, p.ctas * kNP, worker);
   if (cr.g0 >= cr.g1) return;
 
-  Seg seg = first_seg(pre, p.B, H, cr);
+  Seg seg = first_seg<kSlot>(pre, slen, p.B, H, cr);
   if (APPEND) {
     // decode step: append the new token of every (b, h) whose last block
     // this pair owns (only this pair reads that block), before any copy of
     // it is issued; the bulk copies read the cache through the async proxy
-    for (Seg sg = seg; sg.valid; sg = next_seg(sg, pre, p.B, H, cr)) {
+    for (Seg sg = seg; sg.valid; sg = next_seg<kSlot>(sg, pre, slen, p.B, H, cr)) {
       const int raw = p.lengths[sg.b];
-      if (sg.je == sg.nb && raw >= 1 && raw <= p.N_cap)
+      const bool last = kSlot ? (sg.jb < sg.je && sg.je == real_blocks(slen[sg.b])) : (sg.je == sg.nb);
+      if (last && raw >= 1 && raw <= p.N_cap)
         append_tail<BITS, GRP>(p, sg.b, sg.h, raw - 1, (is_s ? 0 : 32) + lane);
     }
     asm volatile("fence.proxy.async;" ::: "memory");
@@ -637,7 +682,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
   // each warp's cursor lives in shared memory and only lane 0 touches it, so
   // it takes no registers in the lanes' loops.
   Prod prod{seg, seg.jb, true};
-  prod = prod_settle(prod, pre, p.B, H, cr);
+  prod = prod_settle<kSlot>(prod, pre, slen, p.B, H, cr);
   static_assert(sizeof(Prod) <= sizeof(unsigned long long) * 6, "cursor slot");
   Prod* cur = reinterpret_cast<Prod*>(ps.cursor[is_s ? 0 : 1]);
   // S-warp: q of a segment, loaded (lane + 32 r) before it is scaled into qs.
@@ -677,7 +722,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
         issue_half<BITS, GRP>(p, ps, s, pr.seg.b, pr.seg.h, pr.j, slen, is_s, extra_tx(is_s));
         ++*issued;
         ++pr.j;
-        pr = prod_settle(pr, pre, p.B, H, cr);
+        pr = prod_settle<kSlot>(pr, pre, slen, p.B, H, cr);
       }
       *cur = pr;
     }
@@ -688,7 +733,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
         ++*issued;
       }
       ++prod.j;
-      prod = prod_settle(prod, pre, p.B, H, cr);
+      prod = prod_settle<kSlot>(prod, pre, slen, p.B, H, cr);
     }
   }
   if (is_s) store_q();
@@ -779,7 +824,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
               issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, true, extra_tx(true));
               ++*issued;
               ++pr.j;
-              *cur = prod_settle(pr, pre, p.B, H, cr);
+              *cur = prod_settle<kSlot>(pr, pre, slen, p.B, H, cr);
             }
           }
         } else if (k > 0 && prod.valid) {
@@ -795,7 +840,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
               ++*issued;
             }
             ++prod.j;
-            prod = prod_settle(prod, pre, p.B, H, cr);
+            prod = prod_settle<kSlot>(prod, pre, slen, p.B, H, cr);
           }
         }
       }
@@ -925,7 +970,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
               issue_half<BITS, GRP>(p, ps, stage, pr.seg.b, pr.seg.h, pr.j, slen, false, 0u);
               ++*issued;
               ++pr.j;
-              *cur = prod_settle(pr, pre, p.B, H, cr);
+              *cur = prod_settle<kSlot>(pr, pre, slen, p.B, H, cr);
             }
           }
         } else if (lane == 0) {
@@ -934,6 +979,11 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       }
 
       if (!alive) break;
+      if (kSlot && seg.jb >= seg.je) {                 // the append slot alone: no state
+        first = false;
+        seg = next_seg<kSlot>(seg, pre, slen, p.B, H, cr);
+        continue;
+      }
       // the pair's state for the segment: z summed over the token lanes, u
       // over the four token groups; lanes with ts = 0 hold channels 16cs..
 #pragma unroll
@@ -941,7 +991,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) z[hh] += __shfl_xor_sync(0xffffffffu, z[hh], o);
       }
-      const bool whole = (seg.jb == 0) && (seg.je == seg.nb) && !p.force_partial;
+      const bool whole = (seg.jb == 0) && (seg.je == seg_blocks<kSlot>(seg, slen)) && !p.force_partial;
       const long long slot = static_cast<long long>(worker) + head;
 #pragma unroll
       for (int hh = 0; hh < kG; ++hh) {
@@ -979,7 +1029,7 @@ __global__ void __launch_bounds__(Tr<BITS, GRP>::kThreads, Tr<BITS, GRP>::kCtasP
       }
     }
     first = false;
-    seg = next_seg(seg, pre, p.B, H, cr);
+    seg = next_seg<kSlot>(seg, pre, slen, p.B, H, cr);
   }
   if (!alive && lane == 0) {
     // a wait ran out: nothing of this pair's segment is written; copies this
@@ -1100,6 +1150,7 @@ kvq_status decode_launch(const AttendArgs& a, cudaStream_t s) {
   m.D = kD;
   m.G = kG;
   m.Lq = 1;
+  m.extra_slots = (a.K_tail_step && a.g.bits == 4) ? 1 : 0;   // the decode kernel's kSlot
   const kvq_status ws = add_window(a, p.partials, static_cast<long long>(partial_slots(m.ctas, a.g.B, a.g.H_kv)),
                                    kG * (kD + 2), kD + 2, 32 * (kD + 2), 1, &m, s);
   if (ws != KVQ_OK) return ws;

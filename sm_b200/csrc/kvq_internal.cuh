@@ -140,6 +140,8 @@ struct MergeArgs {
   int G, Lq;                       // query heads per KV head, rows per query head
   bool feature_major;              // partial layout (rows contiguous per field)
   bool causal;                     // causal rows: a length below Lq leaves rows without keys
+  int extra_slots;                 // per-head plan slots past the last block (the decode step's
+                                   // append, warp_block_prefix's extra); 0 elsewhere
   // recent-token window (kvq_attend_window); win_lengths == nullptr: none.
   // With a window every (b, h) is merged: its window state sits in slot
   // win_slot0 + b * H_kv + h, and no worker wrote an output row itself.

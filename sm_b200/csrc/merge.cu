@@ -62,9 +62,11 @@ __device__ __forceinline__ MergePlan merge_plan(const MergeArgs& a, const int* s
   p.zero = nb == 0 && wl == 0;
   p.win_slot = a.win_slot0 + static_cast<long long>(b) * H + h;
   if (nb > 0) {
+    // nb counts the head's plan slots; its blocks are the first nr of them
+    const int nr = seq_blocks(raw, a.N_cap, a.BT);
     const CtaRange cr = cta_range(s_pre, a.B, H, a.ctas, 0);
     const long long S = static_cast<long long>(H) * s_pre[b] + static_cast<long long>(h) * nb;
-    const long long E = S + nb;
+    const long long E = S + nr;
     p.c_first = S / cr.P;
     p.parts = static_cast<int>((E - 1) / cr.P - p.c_first + 1);
     p.skip = !a.win_lengths && p.parts == 1;
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(kRowMaxWarps * 32) merge_rows_kernel(MergePara
   __shared__ float s_u[kRowMaxWarps][256];
   __shared__ MergePlan s_plan;
   const MergeArgs& a = mp.a;
-  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre, true);
+  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre, true, a.extra_slots);
   const int H = a.H_kv;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(kFmWarps * 32, 5) merge_fm_kernel(MergeParams 
   __shared__ MergePlan s_plan;
   const MergeArgs& a = mp.a;
   const int D = a.D;
-  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre, true);
+  if (threadIdx.x < 32) warp_block_prefix(a.lengths, a.B, a.N_cap, a.BT, s_pre, true, a.extra_slots);
   const int H = a.H_kv;
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh % H;

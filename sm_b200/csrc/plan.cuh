@@ -15,14 +15,22 @@ namespace kvq {
 
 // Warp 0 fills pre[0..B] (the caller synchronises the CTA afterwards).
 // l2: read the lengths at the L2 (ld.global.cg), as a kernel does that reads
-// them before its grid-dependency wait.
+// them before its grid-dependency wait.  extra: slots added per head of every
+// sequence with a length in [1, n_cap] -- the decode step's append, counted
+// as work in the split so the workers that append cover fewer blocks (no
+// block sits in such a slot: a worker's blocks of a head stop at the head's
+// last real block).
 __device__ __forceinline__ void warp_block_prefix(const int32_t* lengths, int B, int n_cap, int bt,
-                                                  int* pre, bool l2 = false) {
+                                                  int* pre, bool l2 = false, int extra = 0) {
   const int lane = threadIdx.x & 31;
   int carry = 0;
   for (int base = 0; base < B; base += 32) {
     const int b = base + lane;
-    int v = b < B ? seq_blocks(l2 ? __ldcg(lengths + b) : __ldg(lengths + b), n_cap, bt) : 0;
+    int v = 0;
+    if (b < B) {
+      const int raw = l2 ? __ldcg(lengths + b) : __ldg(lengths + b);
+      v = seq_blocks(raw, n_cap, bt) + ((raw >= 1 && raw <= n_cap) ? extra : 0);
+    }
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int n = __shfl_up_sync(0xffffffffu, v, o);

@@ -127,3 +127,15 @@ def test_decode_step_bad_length(sm):
         assert torch.equal(a, b_)
     assert torch.all(out == 0)
     sm.check()
+
+
+@pytest.mark.parametrize("bits,steps", [(4, 2), (8, 1)])
+def test_decode_step_full_size(sm, bits, steps):
+    """The decode workload's shape at full size (B 32, H_q 32, H_kv 8, D 128,
+    about 4,096 tokens) in the launch configuration the bench times (automatic
+    splits), every head compared.  With 4-bit codes the split has room to count
+    each appending head's append as one more plan slot (the workers that
+    append cover one block fewer, and some worker ranges start at such a
+    slot); with 8-bit codes it has not, and the plan is the plain one."""
+    start = [4094 - 3 * (b % 4) for b in range(32)]
+    _run_steps(sm, 32, 32, 8, 4096, 128, start, steps, bits, 32, seed=40 + bits)
