@@ -135,6 +135,7 @@ __device__ __forceinline__ void scores_many_rows(float* s_p, const float* s_q, c
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   int d = 0;
   if ((D & 3) == 0) {
+#pragma unroll 8
     for (; d < D; d += 4) {
       const float k0 = kr[d], k1 = kr[d + 1], k2 = kr[d + 2], k3 = kr[d + 3];
 #pragma unroll
@@ -223,17 +224,18 @@ __device__ __forceinline__ void pv_many_rows(float* s_u, const float* s_p, const
     }
 }
 
-// JMAX: features per lane, D <= 32 * JMAX.  One CTA per (b, h_kv, pass of
+// JMAX: features per lane, D <= 32 * JMAX; DC: D when it is fixed at compile
+// time (128), else 0.  One CTA per (b, h_kv, pass of
 // RP rows); the body is a grid-stride loop over the passes, which at this
 // grid runs once (the loop form measured 4 to 8 us faster per step than the
 // same body without it on the decode workload's window).  Two CTAs per SM:
 // the grid of a decode step, B * H_kv CTAs, then fits in one wave.
-template <int JMAX>
+template <int JMAX, int DC>
 __global__ void __launch_bounds__(kWThreads, 2) window_kernel(WindowParams wp) {
   griddep_release();
   const WindowArgs& a = wp.a;
   extern __shared__ float sm[];
-  const int D = a.D, DS = D + 1;
+  const int D = DC ? DC : a.D, DS = D + 1;
   const int R = a.G * a.Lq;
   const int RP = R < kWR ? R : kWR;
   if (RP < 1) {
@@ -374,7 +376,9 @@ kvq_status launch_window(const WindowArgs& w, cudaStream_t s) {
   const long long blocks = static_cast<long long>(w.B) * w.H_kv * (passes < 1 ? 1 : passes);
   if (blocks > 0x7fffffffLL || w.D > 256 || w.D < 1) return KVQ_ERR_UNSUPPORTED;
   const size_t smem = window_smem(w.D, RP);
-  auto kernel = w.D <= 64 ? window_kernel<2> : (w.D <= 128 ? window_kernel<4> : window_kernel<8>);
+  // D = 128 as a compile-time constant: the score loops unroll fully
+  auto kernel = w.D == 128 ? window_kernel<4, 128>
+                           : (w.D <= 64 ? window_kernel<2, 0> : (w.D <= 128 ? window_kernel<4, 0> : window_kernel<8, 0>));
   if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kernel), smem)) return KVQ_ERR_CUDA;
   WindowParams p{w};
   if (launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(kWThreads), smem, s, p) != cudaSuccess)
